@@ -1,0 +1,370 @@
+"""Benchmark of one absorbed-form MLA decode step on B200.
+
+A step is the whole hot path over one batch: mla_cache_append ->
+mla_absorb_q -> mla_decode (decode + split combine) -> mla_out_proj, all
+through the C ABI (libmla.so). Default workload: DeepSeek-V2 dims, batch 64,
+seq_lens ~ U[1024, 8192], paged latent cache (block 64) — the configuration
+the >= 70 % roofline target is stated on. Other workloads: --workload NAME.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+For N > 1 launch under torchrun: every rank runs an independent replica of the
+workload on its own GPU (no data-path collective; "scaling": "weak"); the
+timing is the max over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_latent_kv_33_b200 import synth  # noqa: E402
+
+METRIC = "MLA decode µs/step, latent-cache HBM GB/s and TFLOP/s vs roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="v2_b64_paged", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0, help="target seconds of oracle work")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm --
+
+def upload(x, torch, dev):
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    w = x.w
+    W = {k: bf(v) for k, v in x.weights_bits.items()}
+    cache_t = bf(x.cache)
+    bt = None if x.block_table is None else torch.from_numpy(x.block_table).to(dev)
+    return W, cache_t, bt
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from mla_latent_kv_33_b200 import mla
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        raise SystemExit("bench.py times the bf16 tensor-core workloads")
+    x = synth.generate(w)
+    W, cache_t, bt = upload(x, torch, dev)
+    cache = mla.Cache(cache_t, bt)
+    p = mla.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base, 0.0, w.dtype)
+    T = w.T
+    h = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    pos = torch.from_numpy(x.positions).to(dev)
+    sidx = torch.from_numpy(x.seq_idx).to(dev)
+    sl = torch.from_numpy(x.seq_lens).to(dev)
+    q = torch.empty((T, w.n_h, w.D), device=dev, dtype=torch.bfloat16)
+    o_lat = torch.empty((T, w.n_h, w.d_c), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((T, w.n_h), device=dev, dtype=torch.float32)
+    o = torch.empty((T, w.n_h * w.d_h), device=dev, dtype=torch.bfloat16)
+    ws = {op: torch.empty(max(1, mla.workspace_size(p, op, w.B if op == mla.OP_DECODE else T, w.n_q)),
+                          dtype=torch.uint8, device=dev)
+          for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ)}
+    stream = torch.cuda.current_stream()
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+
+    def step(i=None):
+        mla.mla_cache_append(p, h, W["W_DKV"], W["W_KR"], sidx, pos, cache, ws=ws[mla.OP_APPEND], stream=stream)
+        mla.mla_absorb_q(p, h, W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], pos, q, ws=ws[mla.OP_ABSORB],
+                         stream=stream)
+        if i is not None:
+            ev_dec[i][0].record(stream)
+        mla.mla_decode(p, q, cache, sl, w.n_q, o_lat, lse, ws=ws[mla.OP_DECODE], stream=stream)
+        if i is not None:
+            ev_dec[i][1].record(stream)
+        mla.mla_out_proj(p, o_lat, W["W_UV"], o, ws=ws[mla.OP_OUT_PROJ], stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = mla.mla_get_device_error(stream)
+    if st != mla.MLA_OK:
+        raise RuntimeError(f"device error after warm-up: {mla.status_string(st)}")
+
+    # device-resident timing
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = mla.kernel_launches()
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = mla.kernel_launches() - launches0
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+
+    # end to end through the public API: H2D of the step's inputs from pinned
+    # host memory and D2H of the step's output, inside the timed region
+    h_host = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    pos_host = torch.from_numpy(x.positions).pin_memory()
+    sidx_host = torch.from_numpy(x.seq_idx).pin_memory()
+    sl_host = torch.from_numpy(x.seq_lens).pin_memory()
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = h_host.numel() * 2 + pos_host.numel() * 4 + sidx_host.numel() * 4 + sl_host.numel() * 4
+    d2h = o_host.numel() * 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        h.copy_(h_host, non_blocking=True)
+        pos.copy_(pos_host, non_blocking=True)
+        sidx.copy_(sidx_host, non_blocking=True)
+        sl.copy_(sl_host, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    st = mla.mla_get_device_error(stream)
+    if st != mla.MLA_OK:
+        raise RuntimeError(f"device error during timing: {mla.status_string(st)}")
+
+    step_ms = ms_total / args.steps
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([step_ms, dec_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        step_ms, dec_ms, e2e_ms = (float(v) for v in tt.tolist())
+    return {"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "launches": launches, "clocks": clk.summary(), "x": x, "w": w,
+            "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
+
+
+# ------------------------------------------------------ oracle (CPU) arm --
+
+def oracle_sample(w, x, target_s):
+    """Time the fp64 oracle on a bounded sample of the workload: the whole step
+    for the token rows of a few sequences (append of their new tokens, absorb,
+    decode of all heads over their visible context, W_UV readout). Returns
+    (seconds per step extrapolated by attended-token work, sample text, cores)."""
+    import oracle as orc
+    cores = len(os.sched_getaffinity(0))
+    orc.set_threads(cores)
+    po = orc.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base)
+    oc = orc.Cache(x.cache, x.block_table)
+    work_total = synth.algorithmic_work(w, x.seq_lens)["tokens_attended"]
+    order = np.argsort(x.seq_lens)  # shortest first, grow until the target time
+    done_tokens, seconds, seqs = 0, 0.0, 0
+    t_start = time.perf_counter()
+    for b in order:
+        b = int(b)
+        rows = list(range(b * w.n_q, (b + 1) * w.n_q))
+        t0 = time.perf_counter()
+        orc.append_rows(po, x.h[rows], x.weights["W_DKV"], x.weights["W_KR"], x.positions[rows])
+        qb = orc.absorb_q(po, x.h[rows], x.weights["W_DQ"], x.weights["W_UQ"], x.weights["W_QR"],
+                          x.weights["W_UK"], x.positions[rows])
+        q = np.zeros((w.T, w.n_h, w.D))
+        q[rows] = qb
+        pairs = [(t, hh) for t in rows for hh in range(w.n_h)]
+        o_lat, _ = orc.decode(po, q, oc, x.seq_lens, w.n_q, pairs=pairs)
+        orc.out_proj(po, o_lat.reshape(len(rows), w.n_h, w.d_c), x.weights["W_UV"])
+        seconds += time.perf_counter() - t0
+        done_tokens += sum(int(x.seq_lens[b]) - w.n_q + 1 + j for j in range(w.n_q))
+        seqs += 1
+        if time.perf_counter() - t_start > target_s:
+            break
+    per_step = seconds * work_total / max(1, done_tokens)
+    sample = (f"full step (append, absorb, decode over all {w.n_h} heads, W_UV readout) for {seqs} of "
+              f"{w.B} sequences ({done_tokens} attended tokens of {work_total}); time scaled to the whole "
+              f"batch by attended tokens")
+    return per_step, sample, cores
+
+
+def run_reference(args, rank, world):
+    w = synth.WORKLOADS[args.workload]
+    x = synth.generate(w)
+    per_step_s = []
+    sample_text, cores = "", 0
+    for _ in range(max(1, args.warmup // 3)):
+        oracle_sample(w, x, target_s=min(3.0, args.cpu_sample_s))
+    for _ in range(args.steps):
+        s, sample_text, cores = oracle_sample(w, x, target_s=args.cpu_sample_s / max(1, args.steps))
+        per_step_s.append(s)
+    us = float(np.mean(per_step_s) * 1e6)
+    work = synth.algorithmic_work(w, x.seq_lens)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "µs/step", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args.gpus, x), "gpu_launches": 0,
+        "cpu_baseline": {"value": us, "unit": "µs/step", "cores": cores, "kind": "oracle",
+                         "sample": sample_text},
+        "e2e": {"value": us, "unit": "µs/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cache_gbs": work["cache_bytes"] / (us * 1e-6) / 1e9,
+    }
+    print(json.dumps(line))
+
+
+def config_of(w, n, x):
+    L = x.seq_lens
+    return {"workload": w.name, "description": w.note, "batch": w.B, "n_q": w.n_q,
+            "seq_len_min": int(L.min()), "seq_len_max": int(L.max()), "seq_len_mean": float(L.mean()),
+            "paged": w.paged, "block_size": w.block_size if w.paged else None,
+            "dims": {"d": w.d, "n_h": w.n_h, "d_h": w.d_h, "d_c": w.d_c, "d_cq": w.d_cq, "d_r": w.d_r},
+            "parallelism": f"replicas{n}", "seed": 1000 + w.index,
+            "l2": "no flush: latent cache and weights each exceed the 126 MB L2 (inputs larger than L2)"}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+    finally:
+        pass
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    w, x = r["w"], r["x"]
+    work = synth.algorithmic_work(w, x.seq_lens)
+    peaks, peak_kind = load_peaks()
+    us = r["step_ms"] * 1e3
+    dec_s = r["dec_ms"] * 1e-3
+    cache_gbs = work["cache_bytes"] / dec_s / 1e9
+    tflops = work["flops"] / dec_s / 1e12
+    t_hbm = work["cache_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = work["flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    roof = {
+        "kernel": "mla_decode (k_decode + k_combine)",
+        "bound": bound,
+        "achieved": cache_gbs if bound == "hbm" else tflops,
+        "peak": peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"],
+        "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+        "frac": (t_hbm if bound == "hbm" else t_tc) / dec_s,
+        "traffic": None,
+        "peak_source": peak_kind,
+        "algorithmic_bytes": work["cache_bytes"], "algorithmic_flops": work["flops"],
+        "decode_us": r["dec_ms"] * 1e3,
+        "roofline_us": max(t_hbm, t_tc) * 1e6,
+    }
+    line = {
+        "metric": METRIC, "value": us, "unit": "µs/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world, x),
+        "decode_us": r["dec_ms"] * 1e3, "cache_gbs": cache_gbs, "tflops": tflops,
+        "tokens_per_s": world * w.T / (r["step_ms"] * 1e-3),
+        "roofline": roof,
+        "e2e": {"value": r["e2e_ms"] * 1e3, "unit": "µs/step", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+        "tensor_core_decode": r["tc"],
+        "clocks": r["clocks"],
+    }
+    if not args.no_cpu_baseline and world == 1:
+        s, sample, cores = oracle_sample(w, x, args.cpu_sample_s)
+        line["cpu_baseline"] = {"value": s * 1e6, "unit": "µs/step", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

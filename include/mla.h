@@ -1,0 +1,178 @@
+/*
+ * mla.h — C ABI of libmla.so, the B200 (sm_100a) implementation of the
+ * absorbed-form decode hot path of Multi-head Latent Attention (MLA,
+ * DeepSeek-V2).
+ *
+ * Notation (MLA walk-through, h.sjds.net, section 1; DeepSeek-V2 MLA
+ * explainer, modelers.csdn.net, equations 9-13):
+ *   d     model width (5120 for DeepSeek-V2, 7168 for V3)
+ *   n_h   heads (128), d_h per-head dim (128)
+ *   d_c   KV latent dim (512), d_cq query latent dim d_c' (1536)
+ *   d_r   decoupled RoPE dim d_R (64)
+ *   D     = d_c + d_r, the width of one cached row [c_KV | k_R] (576)
+ *   B     sequences, n_q new tokens per sequence this step, T = B * n_q
+ *         token rows; row t = b * n_q + j holds new token j of sequence b.
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers to tensors are DEVICE pointers unless noted; the caller
+ *     owns every buffer. No entry point allocates or frees device memory.
+ *   - Tensors are dense row-major (C order) with the shapes given below and
+ *     16-byte aligned base addresses (the tensor-memory-accelerator loads
+ *     need it). Element type is the storage dtype of mla_dims.dtype (bf16 or
+ *     fp32) unless stated otherwise; arithmetic accumulates in fp32.
+ *   - Weights are stored out x in, as the pages write them (W_DKV is d_c x d,
+ *     eq. 9; W_UK, W_UV are n_h*d_h x d_c, eqs. 10-11). Head h owns rows
+ *     h*d_h .. h*d_h+d_h-1 of W_UQ, W_UK, W_UV and rows h*d_r .. h*d_r+d_r-1
+ *     of W_QR.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronises, except
+ *     mla_get_device_error.
+ *   - Arguments are validated on the host before any launch; on an invalid
+ *     argument the call returns MLA_ERR_INVALID_ARG (or MLA_ERR_UNSUPPORTED
+ *     for valid but unimplemented shapes) and writes nothing.
+ *     mla_last_error_message() then describes the problem.
+ *   - Contents of device arrays (seq_lens, positions, seq_idx, block tables)
+ *     cannot be checked on the host without a synchronisation. Kernels check
+ *     them and, on a bad value, skip the access, set the library's device
+ *     error word and go on; mla_get_device_error reports it.
+ *   - `ws` is caller-owned device scratch of at least
+ *     mla_workspace_size(...) bytes (may be NULL when that size is 0); it
+ *     must not be shared by calls that run concurrently.
+ *   - A CUDA launch failure returns MLA_ERR_CUDA.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,
+  MLA_ERR_UNSUPPORTED = 2,
+  MLA_ERR_WORKSPACE = 3,
+  MLA_ERR_CUDA = 4,
+  MLA_ERR_TIMEOUT = 5,   /* a kernel's bounded wait expired (device error word) */
+  MLA_ERR_DEVICE_DATA = 6 /* a kernel found an out-of-range index (device error word) */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
+
+/* Layer dimensions. softmax_scale <= 0 selects 1/sqrt(d_h + d_r): the score
+ * of step 4 lives in the (d_h + d_r) = 192-dim concatenation of the content
+ * and position parts (MLA walk-through, section 1 step 4). RoPE uses
+ * RoFormer's interleaved pairs (2i, 2i+1) with theta_i = rope_base^(-2i/d_r). */
+typedef struct {
+  int32_t d, n_h, d_h, d_c, d_cq, d_r;
+  double rope_base;
+  float softmax_scale;
+  int32_t dtype; /* mla_dtype: storage of h, weights, cache, q, o_lat, o */
+} mla_dims;
+
+/* Latent cache (MLA walk-through, section 1 step 1: each token keeps only
+ * [c_KV ; k_R], d_c + d_r numbers, no head label and no K/V split).
+ *   contiguous (paged = 0): data = [num_seqs][max_len][D]; row of
+ *     (b, pos) = b * max_len + pos.
+ *   paged (paged = 1): data = [num_blocks][block_size][D] and block_table =
+ *     [num_seqs][max_blocks_per_seq] int32 (device); row of (b, pos) =
+ *     block_table[b][pos / block_size] * block_size + pos % block_size.
+ * The cache struct itself lives in host memory; data and block_table are
+ * device pointers. */
+typedef struct {
+  void *data;
+  int32_t paged;
+  int32_t block_size;
+  const int32_t *block_table;
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+  int64_t max_len;    /* contiguous only */
+  int64_t num_blocks; /* paged only */
+} mla_cache;
+
+/* Write path (MLA walk-through, section 1 step 1; DeepSeek-V2 explainer,
+ * eq. 9): for every new token row t,
+ *   c_KV = W_DKV h_t  (d_c),  k_R = RoPE(W_KR h_t, positions[t])  (d_r),
+ * rounded once to the storage dtype and stored as the cache row of
+ * (seq_idx[t], positions[t]).
+ *   h         [T][d]            W_DKV [d_c][d]     W_KR [d_r][d]
+ *   seq_idx   [T] int32 device  positions [T] int32 device
+ * A row whose (seq_idx, position) falls outside the cache is not written and
+ * raises MLA_ERR_DEVICE_DATA in the device error word. */
+mla_status mla_cache_append(const mla_dims *dims, const void *h, const void *W_DKV,
+                            const void *W_KR, const int32_t *seq_idx, const int32_t *positions,
+                            int32_t T, const mla_cache *cache, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/* Query path and absorption (MLA walk-through, section 1 step 3 and section
+ * 3 order B; DeepSeek-V2 explainer, eqs. 12-13 and the remark that W_UK can
+ * be absorbed on the query side):
+ *   c_Q = W_DQ h_t (d_cq);  q_C,h = W_UQ_h c_Q (d_h);
+ *   q_R,h = RoPE(W_QR_h c_Q, positions[t]) (d_r);  q_lat,h = W_UK_h^T q_C,h (d_c).
+ *   h [T][d]  W_DQ [d_cq][d]  W_UQ [n_h*d_h][d_cq]  W_QR [n_h*d_r][d_cq]
+ *   W_UK [n_h*d_h][d_c]  positions [T] int32 device
+ *   q (output) [T][n_h][D] = [q_lat | q_R] per head, storage dtype.
+ * c_Q and q_C are tensor-core operands and are rounded to the storage dtype
+ * in the workspace; q is rounded once. */
+mla_status mla_absorb_q(const mla_dims *dims, const void *h, const void *W_DQ, const void *W_UQ,
+                        const void *W_QR, const void *W_UK, const int32_t *positions, int32_t T,
+                        void *q, void *ws, size_t ws_bytes, void *stream);
+
+/* Attention in latent space (MLA walk-through, section 1 step 4 and section
+ * 3 order B): for token row t = b*n_q + j, head h, and every cached position
+ * i < L_b - n_q + 1 + j (L_b = seq_lens[b] counts cached rows after this
+ * step's append; new token j sits at position L_b - n_q + j, causal within
+ * the step):
+ *   s_i = scale * (q_lat,h . c_KV_i + q_R,h . k_R_i),  p = softmax_i(s),
+ *   o_lat[t][h] = sum_i p_i c_KV_i (d_c),  lse[t][h] = log sum_i exp(s_i).
+ *   q [B*n_q][n_h][D]   seq_lens [B] int32 device
+ *   o_lat (output) [B*n_q][n_h][d_c] storage dtype
+ *   lse (output, may be NULL) [B*n_q][n_h] float32 (natural log)
+ * num_splits: 0 = automatic split-KV planning; the tensor-core path always
+ * balances the concatenated KV tiles of all sequences over the GPU and merges
+ * split sequences with a log-sum-exp combine, so only 0 is accepted there.
+ * seq_lens[b] < n_q or beyond the cache capacity raises MLA_ERR_DEVICE_DATA
+ * and that sequence's outputs are left unwritten. */
+mla_status mla_decode(const mla_dims *dims, const void *q, const mla_cache *cache,
+                      const int32_t *seq_lens, int32_t B, int32_t n_q, void *o_lat, float *lse,
+                      int32_t num_splits, void *ws, size_t ws_bytes, void *stream);
+
+/* Per-head readout, decompressed once at the end (MLA walk-through, section
+ * 3 order B; DeepSeek-V2 explainer, eq. 11):
+ *   o[t][h*d_h + i] = sum_j W_UV[h*d_h + i][j] o_lat[t][h][j].
+ *   o_lat [T][n_h][d_c]   W_UV [n_h*d_h][d_c]   o (output) [T][n_h*d_h]. */
+mla_status mla_out_proj(const mla_dims *dims, const void *o_lat, const void *W_UV, int32_t T,
+                        void *o, void *ws, size_t ws_bytes, void *stream);
+
+/* Scratch size in bytes for one call of `op` (MLA_OP_*). `rows` is T for
+ * append/absorb/out_proj and B for decode; n_q and max_seq_len are used by
+ * decode only (max_seq_len may be 0 for the tensor-core path). */
+enum { MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3 };
+size_t mla_workspace_size(const mla_dims *dims, int32_t op, int32_t rows, int32_t n_q,
+                          int64_t max_seq_len);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns MLA_OK, MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_DATA or MLA_ERR_CUDA. */
+mla_status mla_get_device_error(void *stream);
+
+const char *mla_status_string(mla_status s);
+
+/* Text of the last host-side validation or CUDA error on this thread. */
+const char *mla_last_error_message(void);
+
+/* Which kernel family serves a call with these dims: 1 = sm_100a tensor
+ * cores (tcgen05/TMEM/TMA), 0 = CUDA-core kernels (fp32 storage or dims the
+ * tensor-core kernels are not built for). */
+int32_t mla_uses_tensor_cores(const mla_dims *dims, int32_t op);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads). Lets callers count launches inside a timed region. */
+uint64_t mla_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

@@ -1,0 +1,84 @@
+// Shared device helpers of libmla: the device error word, storage-type loads
+// and stores, and RoPE angles.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#define MLA_DEVERR_DATA 1u     // an index from device memory was out of range
+#define MLA_DEVERR_TIMEOUT 2u  // a bounded wait expired
+
+namespace mla {
+
+// One word per device, read and cleared by mla_get_device_error().
+__device__ unsigned int g_dev_error;
+
+__device__ __forceinline__ void dev_error(unsigned int code) { atomicOr(&g_dev_error, code); }
+
+template <typename T>
+__device__ __forceinline__ float ld_f(const T *p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float *p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Pack two floats into one bf16x2 word (round to nearest even), low = a.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// RoPE rotation of the interleaved pair (x0, x1) = (x[2i], x[2i+1]) by the
+// angle pos * base^(-2i/d_r). The angle is formed and reduced in double so
+// positions up to 2^17 and beyond keep full fp32 accuracy.
+__device__ __forceinline__ void rope_pair(float &x0, float &x1, int pair, int d_r, int pos,
+                                          double base) {
+  const double theta = pow(base, -2.0 * static_cast<double>(pair) / static_cast<double>(d_r));
+  double s, c;
+  sincos(static_cast<double>(pos) * theta, &s, &c);
+  const float cf = static_cast<float>(c), sf = static_cast<float>(s);
+  const float y0 = x0 * cf - x1 * sf;
+  const float y1 = x0 * sf + x1 * cf;
+  x0 = y0;
+  x1 = y1;
+}
+
+// Physical cache row of logical (b, pos); returns -1 when out of range.
+struct CacheView {
+  void *data;
+  const int32_t *block_table;
+  int64_t max_len;
+  int64_t num_blocks;
+  int32_t paged;
+  int32_t block_size;
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+};
+
+__device__ __forceinline__ int64_t cache_row(const CacheView &c, int b, int64_t pos) {
+  if (b < 0 || b >= c.num_seqs || pos < 0) return -1;
+  if (!c.paged) return pos < c.max_len ? static_cast<int64_t>(b) * c.max_len + pos : -1;
+  const int64_t blk_idx = pos / c.block_size;
+  if (blk_idx >= c.max_blocks_per_seq) return -1;
+  const int64_t blk = c.block_table[static_cast<int64_t>(b) * c.max_blocks_per_seq + blk_idx];
+  if (blk < 0 || blk >= c.num_blocks) return -1;
+  return blk * c.block_size + pos % c.block_size;
+}
+
+}  // namespace mla

@@ -1,0 +1,430 @@
+// libmla: host side of the C ABI declared in include/mla.h.
+//
+// Validates arguments, sizes workspaces, builds TMA tensor maps and launches
+// the kernels. Two kernel families serve the calls:
+//   - sm_100a tensor-core kernels (tcgen05 MMA into tensor memory, TMA tile
+//     loads, mbarrier pipelines) for bf16 storage at the DeepSeek-V2/V3 head
+//     geometry (n_h = 128, d_h = 128, d_c = 512, d_r = 64);
+//   - CUDA-core kernels for fp32 storage and other dims.
+// mla_uses_tensor_cores() reports which family a call will use; the choice
+// depends only on dims, never on a runtime failure.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <string>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "simt.cuh"
+#include "decode_tc.cuh"
+
+namespace {
+
+thread_local std::string g_msg;
+std::atomic<uint64_t> g_launches{0};
+
+// Every kernel launch goes through this macro so the count is exact.
+#define MLA_LAUNCH(...) (g_launches.fetch_add(1, std::memory_order_relaxed), __VA_ARGS__)
+
+mla_status fail(mla_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+mla_status fail(mla_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return s;
+}
+
+mla_status cuda_check(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(const mla_dims *d) { return d->dtype == MLA_BF16 ? 2 : 4; }
+
+float softmax_scale(const mla_dims *d) {
+  return d->softmax_scale > 0.f ? d->softmax_scale
+                                : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->d_h + d->d_r)));
+}
+
+mla_status check_dims(const mla_dims *d) {
+  if (d == nullptr) return fail(MLA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->d <= 0 || d->n_h <= 0 || d->d_h <= 0 || d->d_c <= 0 || d->d_cq <= 0 || d->d_r <= 0)
+    return fail(MLA_ERR_INVALID_ARG, "all dims must be positive");
+  if (d->d_r % 2 != 0) return fail(MLA_ERR_INVALID_ARG, "d_r must be even (RoPE pairs)");
+  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32)
+    return fail(MLA_ERR_INVALID_ARG, "dtype must be MLA_BF16 or MLA_FP32");
+  if (!(d->rope_base > 1.0)) return fail(MLA_ERR_INVALID_ARG, "rope_base must be > 1");
+  if (d->d_c + d->d_r > 1024)
+    return fail(MLA_ERR_UNSUPPORTED, "d_c + d_r > 1024 is not supported");
+  return MLA_OK;
+}
+
+mla_status check_cache(const mla_cache *c, int D) {
+  (void)D;
+  if (c == nullptr || c->data == nullptr) return fail(MLA_ERR_INVALID_ARG, "cache or cache->data is NULL");
+  if (!aligned16(c->data)) return fail(MLA_ERR_INVALID_ARG, "cache->data must be 16-byte aligned");
+  if (c->num_seqs <= 0) return fail(MLA_ERR_INVALID_ARG, "cache->num_seqs must be positive");
+  if (c->paged) {
+    if (c->block_table == nullptr) return fail(MLA_ERR_INVALID_ARG, "paged cache needs block_table");
+    if (c->block_size <= 0 || c->max_blocks_per_seq <= 0 || c->num_blocks <= 0)
+      return fail(MLA_ERR_INVALID_ARG, "paged cache needs block_size, max_blocks_per_seq, num_blocks > 0");
+  } else if (c->max_len <= 0) {
+    return fail(MLA_ERR_INVALID_ARG, "contiguous cache needs max_len > 0");
+  }
+  return MLA_OK;
+}
+
+mla::CacheView view_of(const mla_cache *c) {
+  mla::CacheView v;
+  v.data = c->data;
+  v.block_table = c->block_table;
+  v.max_len = c->max_len;
+  v.num_blocks = c->num_blocks;
+  v.paged = c->paged;
+  v.block_size = c->block_size;
+  v.max_blocks_per_seq = c->max_blocks_per_seq;
+  v.num_seqs = c->num_seqs;
+  return v;
+}
+
+bool tc_geometry(const mla_dims *d) {
+  return d->dtype == MLA_BF16 && d->n_h == 128 && d->d_h == 128 && d->d_c == 512 && d->d_r == 64 &&
+         d->d % 64 == 0 && d->d_cq % 64 == 0;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------ CUDA-core variants --
+
+template <typename T>
+void launch_linear(const T *W, int64_t w_sb, int64_t w_sn, int64_t w_sk, const void *X, bool x_fp32,
+                   int64_t x_sb, int64_t x_st, float *Y, int64_t y_sb, int64_t y_st, int N, int K, int Tn,
+                   int batches, cudaStream_t st) {
+  dim3 grid((N + 7) / 8, Tn, batches);
+  if (x_fp32)
+    MLA_LAUNCH(mla::k_simt_linear<T, float><<<grid, 256, 0, st>>>(W, w_sb, w_sn, w_sk, static_cast<const float *>(X),
+                                                       x_sb, x_st, Y, y_sb, y_st, N, K));
+  else
+    MLA_LAUNCH(mla::k_simt_linear<T, T><<<grid, 256, 0, st>>>(W, w_sb, w_sn, w_sk, static_cast<const T *>(X), x_sb,
+                                                   x_st, Y, y_sb, y_st, N, K));
+}
+
+template <typename T>
+mla_status simt_append(const mla_dims *d, const void *h, const void *W_DKV, const void *W_KR,
+                       const int32_t *seq_idx, const int32_t *positions, int Tn, const mla_cache *c,
+                       void *ws, cudaStream_t st) {
+  const int D = d->d_c + d->d_r;
+  float *rows = static_cast<float *>(ws);  // [T][D] = [W_DKV h_t | W_KR h_t]
+  launch_linear<T>(static_cast<const T *>(W_DKV), 0, d->d, 1, h, false, 0, d->d, rows, 0, D, d->d_c, d->d,
+                   Tn, 1, st);
+  launch_linear<T>(static_cast<const T *>(W_KR), 0, d->d, 1, h, false, 0, d->d, rows + d->d_c, 0, D, d->d_r,
+                   d->d, Tn, 1, st);
+  MLA_LAUNCH(mla::k_simt_append_store<T><<<Tn, 128, 0, st>>>(rows, D, d->d_c, d->d_r, d->rope_base, seq_idx,
+                                                  positions, view_of(c)));
+  return cuda_check("append (CUDA cores)");
+}
+
+size_t simt_append_ws(const mla_dims *d, int Tn) {
+  return sizeof(float) * static_cast<size_t>(Tn) * (d->d_c + d->d_r);
+}
+
+template <typename T>
+mla_status simt_absorb(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ,
+                       const void *W_QR, const void *W_UK, const int32_t *positions, int Tn, void *q,
+                       void *ws, cudaStream_t st) {
+  const int64_t HD = static_cast<int64_t>(d->n_h) * d->d_h;
+  const int64_t HR = static_cast<int64_t>(d->n_h) * d->d_r;
+  const int64_t HC = static_cast<int64_t>(d->n_h) * d->d_c;
+  float *cq = static_cast<float *>(ws);          // [T][d_cq]
+  float *qc = cq + static_cast<int64_t>(Tn) * d->d_cq;  // [T][n_h*d_h]
+  float *qr = qc + Tn * HD;                      // [T][n_h*d_r]
+  float *ql = qr + Tn * HR;                      // [T][n_h][d_c]
+  launch_linear<T>(static_cast<const T *>(W_DQ), 0, d->d, 1, h, false, 0, d->d, cq, 0, d->d_cq, d->d_cq, d->d,
+                   Tn, 1, st);
+  launch_linear<T>(static_cast<const T *>(W_UQ), 0, d->d_cq, 1, cq, true, 0, d->d_cq, qc, 0, HD,
+                   static_cast<int>(HD), d->d_cq, Tn, 1, st);
+  launch_linear<T>(static_cast<const T *>(W_QR), 0, d->d_cq, 1, cq, true, 0, d->d_cq, qr, 0, HR,
+                   static_cast<int>(HR), d->d_cq, Tn, 1, st);
+  // q_lat,h[j] = sum_i W_UK[h*d_h + i][j] q_C,h[i]: batch = head, W(h, n=j, k=i)
+  launch_linear<T>(static_cast<const T *>(W_UK), static_cast<int64_t>(d->d_h) * d->d_c, 1, d->d_c, qc, true,
+                   d->d_h, HD, ql, d->d_c, HC, d->d_c, d->d_h, Tn, d->n_h, st);
+  MLA_LAUNCH(mla::k_simt_q_store<T><<<Tn * d->n_h, 128, 0, st>>>(ql, qr, d->n_h, d->d_c, d->d_r, d->rope_base,
+                                                      positions, static_cast<T *>(q)));
+  return cuda_check("absorb (CUDA cores)");
+}
+
+size_t simt_absorb_ws(const mla_dims *d, int Tn) {
+  const size_t t = static_cast<size_t>(Tn);
+  return sizeof(float) * t * (d->d_cq + static_cast<size_t>(d->n_h) * (d->d_h + d->d_r + d->d_c));
+}
+
+template <typename T>
+mla_status simt_decode(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int B,
+                       int n_q, void *o_lat, float *lse, cudaStream_t st) {
+  const int rows = B * n_q * d->n_h;
+  const size_t smem = sizeof(float) * 8 * d->d_c;
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(mla::k_simt_decode<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+  MLA_LAUNCH(mla::k_simt_decode<T><<<rows, 256, smem, st>>>(static_cast<const T *>(q), view_of(c), seq_lens, n_q,
+                                                 d->n_h, d->d_c, d->d_r, softmax_scale(d),
+                                                 static_cast<T *>(o_lat), lse));
+  return cuda_check("decode (CUDA cores)");
+}
+
+template <typename T>
+mla_status simt_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int Tn, void *o, void *ws,
+                         cudaStream_t st) {
+  // o[t][h*d_h + i] = sum_j W_UV[h*d_h+i][j] o_lat[t][h][j]: batch = head
+  const int64_t HD = static_cast<int64_t>(d->n_h) * d->d_h;
+  float *y = static_cast<float *>(ws);  // [T][n_h*d_h]
+  launch_linear<T>(static_cast<const T *>(W_UV), static_cast<int64_t>(d->d_h) * d->d_c, d->d_c, 1, o_lat,
+                   false, d->d_c, static_cast<int64_t>(d->n_h) * d->d_c, y, d->d_h, HD, d->d_h, d->d_c, Tn,
+                   d->n_h, st);
+  const int64_t n = Tn * HD;
+  const int64_t blocks = (n + 255) / 256;
+  MLA_LAUNCH(mla::k_simt_store<T><<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(y, static_cast<T *>(o), n));
+  return cuda_check("out_proj (CUDA cores)");
+}
+
+size_t simt_out_proj_ws(const mla_dims *d, int Tn) {
+  return sizeof(float) * static_cast<size_t>(Tn) * d->n_h * d->d_h;
+}
+
+
+// ------------------------------------------------------------- TMA maps --
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void *ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer][inner] array with row pitch
+// `pitch_bytes`, box [box_outer][box_inner], 128-byte swizzle.
+mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
+                          uint32_t box_inner, uint32_t box_outer, const char *what) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "tensor map for %s: CUresult %d", what, static_cast<int>(r));
+  return MLA_OK;
+}
+
+// ------------------------------------------------- tensor-core decode ----
+
+mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int B, int n_q,
+                     void *o_lat, float *lse, void *ws, size_t ws_bytes, cudaStream_t st) {
+  namespace D = mla::dec;
+  const int BJ = B * n_q;
+  if (BJ > D::MAX_UNITS) return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode supports B*n_q <= %d", D::MAX_UNITS);
+  if (c->paged && c->block_size % D::TILE != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode needs block_size to be a multiple of %d", D::TILE);
+  const int64_t rows = c->paged ? c->num_blocks * c->block_size : static_cast<int64_t>(c->num_seqs) * c->max_len;
+  if (rows >= 0x7fff0000LL) return fail(MLA_ERR_UNSUPPORTED, "cache has too many rows for 32-bit TMA coordinates");
+  const int sms = sm_count();
+  const int nclusters = sms / 2;
+  if (ws_bytes < mla::decode_tc_ws(B, n_q, sms)) return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
+
+  CUtensorMap tm_q, tm_ks, tm_v;
+  mla_status s;
+  if ((s = make_tmap_bf16(&tm_q, q, D::D, static_cast<uint64_t>(BJ) * D::HEADS, D::D * 2, 64, D::HPC, "q")) != MLA_OK)
+    return s;
+  if ((s = make_tmap_bf16(&tm_ks, c->data, D::D, rows, D::D * 2, 64, D::OWN, "cache (score tile)")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tm_v, c->data, D::D, rows, D::D * 2, 64, D::TILE, "cache (value tile)")) != MLA_OK) return s;
+
+  D::Params p{};
+  p.seq_lens = seq_lens;
+  p.block_table = c->block_table;
+  p.max_len = c->max_len;
+  p.cache_rows = rows;
+  p.paged = c->paged;
+  p.block_size = c->block_size;
+  p.max_blocks_per_seq = c->max_blocks_per_seq;
+  p.num_blocks_i32 = static_cast<int32_t>(c->paged ? c->num_blocks : 0);
+  p.B = B;
+  p.n_q = n_q;
+  p.capacity = c->paged ? static_cast<int64_t>(c->max_blocks_per_seq) * c->block_size : c->max_len;
+  p.scale = softmax_scale(d);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.o_lat = static_cast<__nv_bfloat16 *>(o_lat);
+  p.lse = lse;
+  const size_t plan_bytes = ((static_cast<size_t>(BJ) + 3) * sizeof(int32_t) + 255) & ~size_t(255);
+  const size_t slots = static_cast<size_t>(BJ) + nclusters;
+  p.plan = static_cast<int32_t *>(ws);
+  p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan_bytes);
+  p.part_lse = p.part_o + slots * D::HEADS * D::DC;
+
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(D::k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES) != cudaSuccess)
+      return cuda_check("decode: set shared memory size");
+    attr_done = true;
+  }
+  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_ks, tm_v, p));
+  if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
+  MLA_LAUNCH(D::k_combine<<<BJ * 16, 256, 0, st>>>(p));
+  return cuda_check("decode combine");
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------- C ABI --
+
+extern "C" {
+
+const char *mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+    case MLA_ERR_DEVICE_DATA: return "MLA_ERR_DEVICE_DATA";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+const char *mla_last_error_message(void) { return g_msg.c_str(); }
+
+uint64_t mla_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
+  if (d == nullptr || !tc_geometry(d)) return 0;
+  return op == MLA_OP_DECODE ? 1 : 0;
+}
+
+size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len) {
+  (void)max_seq_len;
+  if (d == nullptr || rows <= 0) return 0;
+  const bool tc = tc_geometry(d);
+  switch (op) {
+    case MLA_OP_APPEND: return simt_append_ws(d, rows);
+    case MLA_OP_ABSORB: return simt_absorb_ws(d, rows);
+    case MLA_OP_DECODE: return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count()) : 0;
+    case MLA_OP_OUT_PROJ: return simt_out_proj_ws(d, rows);
+  }
+  return 0;
+}
+
+mla_status mla_get_device_error(void *stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, mla::g_dev_error, sizeof word);
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "read device error word: %s", cudaGetErrorString(e));
+  e = cudaMemcpyToSymbol(mla::g_dev_error, &zero, sizeof zero);
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "clear device error word: %s", cudaGetErrorString(e));
+  if (word & MLA_DEVERR_TIMEOUT) return fail(MLA_ERR_TIMEOUT, "a kernel's bounded wait expired");
+  if (word & MLA_DEVERR_DATA) return fail(MLA_ERR_DEVICE_DATA, "a kernel found an out-of-range index in device data");
+  return MLA_OK;
+}
+
+mla_status mla_cache_append(const mla_dims *d, const void *h, const void *W_DKV, const void *W_KR,
+                            const int32_t *seq_idx, const int32_t *positions, int32_t T, const mla_cache *c,
+                            void *ws, size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!h || !W_DKV || !W_KR || !seq_idx || !positions)
+    return fail(MLA_ERR_INVALID_ARG, "append: NULL tensor argument");
+  if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(W_KR))
+    return fail(MLA_ERR_INVALID_ARG, "append: h and weights must be 16-byte aligned");
+  if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
+  const size_t need = mla_workspace_size(d, MLA_OP_APPEND, T, 1, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "append needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == MLA_BF16)
+    return simt_append<__nv_bfloat16>(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
+  return simt_append<float>(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
+}
+
+mla_status mla_absorb_q(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                        const void *W_UK, const int32_t *positions, int32_t T, void *q, void *ws, size_t ws_bytes,
+                        void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!h || !W_DQ || !W_UQ || !W_QR || !W_UK || !positions || !q)
+    return fail(MLA_ERR_INVALID_ARG, "absorb: NULL tensor argument");
+  if (!aligned16(h) || !aligned16(W_DQ) || !aligned16(W_UQ) || !aligned16(W_QR) || !aligned16(W_UK) ||
+      !aligned16(q))
+    return fail(MLA_ERR_INVALID_ARG, "absorb: tensors must be 16-byte aligned");
+  const size_t need = mla_workspace_size(d, MLA_OP_ABSORB, T, 1, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "absorb needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == MLA_BF16)
+    return simt_absorb<__nv_bfloat16>(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
+  return simt_absorb<float>(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
+}
+
+mla_status mla_decode(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int32_t B,
+                      int32_t n_q, void *o_lat, float *lse, int32_t num_splits, void *ws, size_t ws_bytes,
+                      void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (B <= 0 || n_q <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_q must be positive");
+  if (!q || !seq_lens || !o_lat) return fail(MLA_ERR_INVALID_ARG, "decode: NULL tensor argument");
+  if (!aligned16(q) || !aligned16(o_lat)) return fail(MLA_ERR_INVALID_ARG, "decode: q and o_lat must be 16-byte aligned");
+  if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
+  if (B > c->num_seqs) return fail(MLA_ERR_INVALID_ARG, "B exceeds cache->num_seqs");
+  if (num_splits < 0) return fail(MLA_ERR_INVALID_ARG, "num_splits must be >= 0");
+  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "decode needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) {
+    if (num_splits != 0)
+      return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode plans its own splits: pass num_splits = 0");
+    return decode_tc(d, q, c, seq_lens, B, n_q, o_lat, lse, ws, ws_bytes, st);
+  }
+  if (d->dtype == MLA_BF16) return simt_decode<__nv_bfloat16>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
+  return simt_decode<float>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
+}
+
+mla_status mla_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int32_t T, void *o, void *ws,
+                        size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!o_lat || !W_UV || !o) return fail(MLA_ERR_INVALID_ARG, "out_proj: NULL tensor argument");
+  if (!aligned16(o_lat) || !aligned16(W_UV) || !aligned16(o))
+    return fail(MLA_ERR_INVALID_ARG, "out_proj: tensors must be 16-byte aligned");
+  const size_t need = mla_workspace_size(d, MLA_OP_OUT_PROJ, T, 1, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "out_proj needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == MLA_BF16) return simt_out_proj<__nv_bfloat16>(d, o_lat, W_UV, T, o, ws, st);
+  return simt_out_proj<float>(d, o_lat, W_UV, T, o, ws, st);
+}
+
+}  // extern "C"

@@ -236,3 +236,59 @@ def algorithmic_work(w: Workload, seq_lens: np.ndarray) -> dict:
         "flops": vis * w.n_h * 2 * (w.D + w.d_c),
         "tokens_attended": vis,
     }
+
+
+@dataclass
+class DecodeInputs:
+    w: Workload
+    q: np.ndarray                     # [T][n_h][D] float32 storage-exact
+    q_bits: np.ndarray | None
+    seq_lens: np.ndarray
+    cache: np.ndarray
+    block_table: np.ndarray | None
+
+
+def generate_decode(w: Workload, seed: int, seq_lens=None, q_scale: float = 0.5) -> DecodeInputs:
+    """Inputs of the decode step alone: absorbed queries drawn directly
+    (q_lat ~ N(0, q_scale^2), q_R ~ N(0, 1): the spread the absorb step gives
+    under the weight scaling above) and a cache of N(0, 1) rows, NaN canaries
+    in unused slots. seq_lens (optional) overrides the workload's length recipe."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if seq_lens is None:
+        seq_lens = _lengths(w, rng)
+    seq_lens = np.asarray(seq_lens, np.int32)
+    w = replace(w, B=len(seq_lens))
+    qv = rng.standard_normal((w.T, w.n_h, w.D), dtype=np.float32)
+    qv[:, :, : w.d_c] *= np.float32(q_scale)
+    q, q_bits = _round_store(qv, w.dtype)
+    B, D = w.B, w.D
+    block_table = None
+    if w.paged:
+        bs = w.block_size
+        nblk = (seq_lens.astype(np.int64) + bs - 1) // bs
+        total = int(nblk.sum())
+        perm = rng.permutation(total).astype(np.int32)
+        block_table = np.zeros((B, int(nblk.max())), np.int32)
+        off = 0
+        for b in range(B):
+            block_table[b, : nblk[b]] = perm[off: off + nblk[b]]
+            off += int(nblk[b])
+        shape = (total, bs, D)
+    else:
+        shape = (B, int(seq_lens.max()), D)
+    nrows = shape[0] * shape[1]
+    if w.dtype == "bf16":
+        cache = np.full((nrows, D), BF16_NAN, np.uint16)
+    else:
+        cache = np.full((nrows, D), F32_NAN_BITS, np.uint32).view(np.float32)
+    for b in range(B):
+        n = int(seq_lens[b])
+        vals = rng.standard_normal((n, D), dtype=np.float32)
+        stored, bits = _round_store(vals, w.dtype)
+        pos = np.arange(n, dtype=np.int64)
+        if w.paged:
+            rows = block_table[b, pos // w.block_size].astype(np.int64) * w.block_size + pos % w.block_size
+        else:
+            rows = np.int64(b) * shape[1] + pos
+        cache[rows] = bits if bits is not None else stored
+    return DecodeInputs(w, q, q_bits, seq_lens, cache.reshape(shape), block_table)
