@@ -16,6 +16,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <string>
 
@@ -23,6 +24,7 @@
 #include "common.cuh"
 #include "ptx.cuh"
 #include "simt.cuh"
+#include "gemm_tc.cuh"
 #include "decode_tc.cuh"
 
 namespace {
@@ -225,9 +227,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 tensor map over a row-major [outer][inner] array with row pitch
-// `pitch_bytes`, box [box_outer][box_inner], 128-byte swizzle.
+// `pitch_bytes`, box [box_outer][box_inner], 128-byte swizzle. Encoded maps
+// are kept in a small per-thread cache keyed by all of their arguments.
+struct TmapKey {
+  const void *base;
+  uint64_t inner, outer, pitch;
+  uint32_t bi, bo;
+  bool operator==(const TmapKey &o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && pitch == o.pitch && bi == o.bi && bo == o.bo;
+  }
+};
+
 mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
                           uint32_t box_inner, uint32_t box_outer, const char *what) {
+  constexpr int CAP = 64;
+  thread_local TmapKey keys[CAP];
+  thread_local CUtensorMap maps[CAP];
+  thread_local int used = 0, next = 0;
+  const TmapKey key{base, inner, outer, pitch_bytes, box_inner, box_outer};
+  for (int i = 0; i < used; ++i)
+    if (keys[i] == key) {
+      *m = maps[i];
+      return MLA_OK;
+    }
   auto fn = encode_fn();
   if (fn == nullptr) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, outer};
@@ -238,10 +260,187 @@ mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "tensor map for %s: CUresult %d", what, static_cast<int>(r));
+  keys[next] = key;
+  maps[next] = *m;
+  next = (next + 1) % CAP;
+  if (used < CAP) ++used;
   return MLA_OK;
 }
 
+// ------------------------------------------------ tensor-core projections --
+
+namespace G = mla::gemm;
+
+struct GemmShape {
+  int m_total, m_tiles, n_tile, n_tiles, k_blocks, splits, batches;
+};
+
+GemmShape gemm_shape(int m_total, int T, int K, int batches) {
+  GemmShape g;
+  g.m_total = m_total;
+  g.m_tiles = (m_total + G::BM - 1) / G::BM;
+  g.n_tile = G::n_tile_for(T);
+  g.n_tiles = (T + g.n_tile - 1) / g.n_tile;
+  g.k_blocks = K / G::BK;
+  g.batches = batches;
+  g.splits = G::choose_splits(g.m_tiles * g.n_tiles * batches, g.k_blocks, sm_count());
+  return g;
+}
+
+size_t gemm_part_bytes(const GemmShape &g, int T) {
+  return sizeof(float) * static_cast<size_t>(g.batches) * g.splits * T * g.m_total;
+}
+
+mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const GemmShape &g,
+                       int T, int m_split, bool a_mn_major, int a_batch_rows, int b_batch_cols, float *out,
+                       cudaStream_t st) {
+  G::Params p{};
+  p.m_total = g.m_total;
+  p.m_split = m_split;
+  p.n_total = T;
+  p.n_tile = g.n_tile;
+  p.k_total = g.k_blocks * G::BK;
+  p.k_blocks_per_split = (g.k_blocks + g.splits - 1) / g.splits;
+  p.splits = g.splits;
+  p.a_mn_major = a_mn_major ? 1 : 0;
+  p.a_batch_rows = a_batch_rows;
+  p.b_batch_cols = b_batch_cols;
+  p.stages = G::stages_for(g.n_tile);
+  p.out = out;
+  const size_t smem = G::smem_for(g.n_tile, p.stages);
+  static size_t attr = 0;
+  if (smem > attr) {
+    if (cudaFuncSetAttribute(G::k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
+      return cuda_check("gemm: set shared memory size");
+    attr = 232448;
+  }
+  dim3 grid(g.m_tiles, g.n_tiles, g.batches * g.splits);
+  MLA_LAUNCH(G::k_gemm<<<grid, G::NUM_THREADS, smem, st>>>(ta, ta2, tb, p));
+  return cuda_check("projection GEMM (tensor cores)");
+}
+
+GemmShape append_shape(const mla_dims *d, int T) { return gemm_shape(d->d_c + d->d_r, T, d->d, 1); }
+
+size_t tc_append_ws(const mla_dims *d, int T) { return gemm_part_bytes(append_shape(d, T), T); }
+
+mla_status tc_append(const mla_dims *d, const void *h, const void *W_DKV, const void *W_KR, const int32_t *seq_idx,
+                     const int32_t *positions, int T, const mla_cache *c, void *ws, cudaStream_t st) {
+  const GemmShape g = append_shape(d, T);
+  CUtensorMap ta, ta2, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_DKV, d->d, d->d_c, d->d * 2ull, 64, 128, "W_DKV")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&ta2, W_KR, d->d, d->d_r, d->d * 2ull, 64, 128, "W_KR")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, g.n_tile, "h")) != MLA_OK) return s;
+  float *part = static_cast<float *>(ws);
+  if ((s = launch_gemm(ta, ta2, tb, g, T, d->d_c, false, 0, 0, part, st)) != MLA_OK) return s;
+  MLA_LAUNCH(G::k_fin_append<<<T, 288, 0, st>>>(part, g.splits, T, d->d_c, d->d_r, d->rope_base, seq_idx, positions,
+                                               view_of(c)));
+  return cuda_check("append finalize");
+}
+
+struct AbsorbPlan {
+  GemmShape cq, uq, uk;
+  size_t part, cq_off, qc_off, total;
+};
+
+AbsorbPlan absorb_plan(const mla_dims *d, int T) {
+  AbsorbPlan a;
+  a.cq = gemm_shape(d->d_cq, T, d->d, 1);
+  a.uq = gemm_shape(d->n_h * (d->d_h + d->d_r), T, d->d_cq, 1);
+  a.uk = gemm_shape(d->d_c, T, d->d_h, d->n_h);
+  size_t part = gemm_part_bytes(a.cq, T);
+  part = std::max(part, gemm_part_bytes(a.uq, T));
+  part = std::max(part, gemm_part_bytes(a.uk, T));
+  a.part = (part + 255) & ~size_t(255);
+  a.cq_off = a.part;
+  a.qc_off = a.cq_off + ((static_cast<size_t>(T) * d->d_cq * 2 + 255) & ~size_t(255));
+  a.total = a.qc_off + static_cast<size_t>(T) * d->n_h * d->d_h * 2;
+  return a;
+}
+
+size_t tc_absorb_ws(const mla_dims *d, int T) { return absorb_plan(d, T).total; }
+
+mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                     const void *W_UK, const int32_t *positions, int T, void *q, void *ws, cudaStream_t st) {
+  const AbsorbPlan a = absorb_plan(d, T);
+  float *part = static_cast<float *>(ws);
+  __nv_bfloat16 *cq = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.cq_off);
+  __nv_bfloat16 *qc = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.qc_off);
+  const int HD = d->n_h * d->d_h;
+  CUtensorMap ta, ta2, tb;
+  mla_status s;
+  // c_Q = W_DQ h
+  if ((s = make_tmap_bf16(&ta, W_DQ, d->d, d->d_cq, d->d * 2ull, 64, 128, "W_DQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, a.cq.n_tile, "h")) != MLA_OK) return s;
+  if ((s = launch_gemm(ta, ta, tb, a.cq, T, d->d_cq, false, 0, 0, part, st)) != MLA_OK) return s;
+  MLA_LAUNCH(G::k_fin_store<<<std::max(1, std::min(1024, T * d->d_cq / 512)), 256, 0, st>>>(part, a.cq.splits, T,
+                                                                                         d->d_cq, cq, d->d_cq));
+  // [q_C ; q_R] = [W_UQ ; W_QR] c_Q, RoPE on q_R
+  if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&ta2, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK)
+    return s;
+  if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, a.uq.n_tile, "c_Q")) != MLA_OK) return s;
+  if ((s = launch_gemm(ta, ta2, tb, a.uq, T, HD, false, 0, 0, part, st)) != MLA_OK) return s;
+  MLA_LAUNCH(G::k_fin_uq<<<dim3(24, T), 512, 0, st>>>(part, a.uq.splits, T, d->n_h, d->d_h, d->d_c, d->d_r,
+                                                     d->rope_base, positions, qc, static_cast<__nv_bfloat16 *>(q)));
+  // q_lat,h = W_UK_h^T q_C,h: A(m = latent j, k = i) = W_UK[h*d_h + i][j], m contiguous
+  if ((s = make_tmap_bf16(&ta, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UK")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, qc, HD, T, HD * 2ull, 64, a.uk.n_tile, "q_C")) != MLA_OK) return s;
+  if ((s = launch_gemm(ta, ta, tb, a.uk, T, d->d_c, true, d->d_h, d->d_h, part, st)) != MLA_OK) return s;
+  const int64_t D = d->d_c + d->d_r;
+  MLA_LAUNCH(G::k_fin_heads<<<dim3(std::max(1, std::min(64, T * d->d_c / 512)), d->n_h), 256, 0, st>>>(
+      part, a.uk.splits, T, d->d_c, d->n_h, static_cast<__nv_bfloat16 *>(q), d->n_h * D, D));
+  return cuda_check("absorb finalize");
+}
+
+GemmShape out_proj_shape(const mla_dims *d, int T) { return gemm_shape(d->d_h, T, d->d_c, d->n_h); }
+
+size_t tc_out_proj_ws(const mla_dims *d, int T) { return gemm_part_bytes(out_proj_shape(d, T), T); }
+
+mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int T, void *o, void *ws,
+                       cudaStream_t st) {
+  const GemmShape g = out_proj_shape(d, T);
+  const int HD = d->n_h * d->d_h, HC = d->n_h * d->d_c;
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_UV, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UV")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, o_lat, HC, T, HC * 2ull, 64, g.n_tile, "o_lat")) != MLA_OK) return s;
+  float *part = static_cast<float *>(ws);
+  if ((s = launch_gemm(ta, ta, tb, g, T, d->d_h, false, d->d_h, d->d_c, part, st)) != MLA_OK) return s;
+  MLA_LAUNCH(G::k_fin_heads<<<dim3(std::max(1, std::min(64, T * d->d_h / 512)), d->n_h), 256, 0, st>>>(
+      part, g.splits, T, d->d_h, d->n_h, static_cast<__nv_bfloat16 *>(o), HD, d->d_h));
+  return cuda_check("out_proj finalize");
+}
+
 // ------------------------------------------------- tensor-core decode ----
+
+// Clusters of two CTAs that can be resident at once (a pair must share a GPC,
+// so this can be below SMs / 2). The persistent decode grid uses exactly this
+// many so that no cluster waits for a second wave.
+int decode_clusters(int sms) {
+  static int cached = 0;
+  if (cached > 0) return cached;
+  namespace D = mla::dec;
+  cudaFuncSetAttribute(D::k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+  cfg.blockDim = dim3(D::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = D::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, D::k_decode, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sms / 2;
+  }
+  cached = std::min(n, sms / 2);
+  return cached;
+}
 
 mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int B, int n_q,
                      void *o_lat, float *lse, void *ws, size_t ws_bytes, cudaStream_t st) {
@@ -253,7 +452,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   const int64_t rows = c->paged ? c->num_blocks * c->block_size : static_cast<int64_t>(c->num_seqs) * c->max_len;
   if (rows >= 0x7fff0000LL) return fail(MLA_ERR_UNSUPPORTED, "cache has too many rows for 32-bit TMA coordinates");
   const int sms = sm_count();
-  const int nclusters = sms / 2;
+  const int nclusters = decode_clusters(sms);
   if (ws_bytes < mla::decode_tc_ws(B, n_q, sms)) return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
 
   CUtensorMap tm_q, tm_ks, tm_v;
@@ -322,7 +521,7 @@ uint64_t mla_kernel_launches(void) { return g_launches.load(std::memory_order_re
 
 int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   if (d == nullptr || !tc_geometry(d)) return 0;
-  return op == MLA_OP_DECODE ? 1 : 0;
+  return (op >= MLA_OP_APPEND && op <= MLA_OP_OUT_PROJ) ? 1 : 0;
 }
 
 size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len) {
@@ -330,10 +529,10 @@ size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n
   if (d == nullptr || rows <= 0) return 0;
   const bool tc = tc_geometry(d);
   switch (op) {
-    case MLA_OP_APPEND: return simt_append_ws(d, rows);
-    case MLA_OP_ABSORB: return simt_absorb_ws(d, rows);
+    case MLA_OP_APPEND: return tc ? tc_append_ws(d, rows) : simt_append_ws(d, rows);
+    case MLA_OP_ABSORB: return tc ? tc_absorb_ws(d, rows) : simt_absorb_ws(d, rows);
     case MLA_OP_DECODE: return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count()) : 0;
-    case MLA_OP_OUT_PROJ: return simt_out_proj_ws(d, rows);
+    case MLA_OP_OUT_PROJ: return tc ? tc_out_proj_ws(d, rows) : simt_out_proj_ws(d, rows);
   }
   return 0;
 }
@@ -365,6 +564,7 @@ mla_status mla_cache_append(const mla_dims *d, const void *h, const void *W_DKV,
   const size_t need = mla_workspace_size(d, MLA_OP_APPEND, T, 1, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "append needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_append(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
   if (d->dtype == MLA_BF16)
     return simt_append<__nv_bfloat16>(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
   return simt_append<float>(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
@@ -384,6 +584,7 @@ mla_status mla_absorb_q(const mla_dims *d, const void *h, const void *W_DQ, cons
   const size_t need = mla_workspace_size(d, MLA_OP_ABSORB, T, 1, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "absorb needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_absorb(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
   if (d->dtype == MLA_BF16)
     return simt_absorb<__nv_bfloat16>(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
   return simt_absorb<float>(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
@@ -423,6 +624,7 @@ mla_status mla_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, 
   const size_t need = mla_workspace_size(d, MLA_OP_OUT_PROJ, T, 1, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "out_proj needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_out_proj(d, o_lat, W_UV, T, o, ws, st);
   if (d->dtype == MLA_BF16) return simt_out_proj<__nv_bfloat16>(d, o_lat, W_UV, T, o, ws, st);
   return simt_out_proj<float>(d, o_lat, W_UV, T, o, ws, st);
 }
