@@ -6,27 +6,45 @@
 //   positions i, p = softmax(s), o_lat = sum_i p_i c_KV_i, lse = log sum exp s.
 //
 // Design (B200, one GPU):
-//  * All 128 heads of a token row share every cached row, so per 64-token
-//    tile S = Q K^T is a dense 128 x 64 x 576 contraction and O += P V a dense
-//    128 x 512 x 64 one. Both run as tcgen05.mma.cta_group::2 on a pair of
-//    SMs (a 2-CTA cluster): CTA r holds heads 64r..64r+63 of Q, its half of
-//    the tile's tokens for QK^T (B operand split by N = tokens) and all 64
-//    tokens of its 256 latent columns for PV (B operand split by N = latent).
-//    The 128 x 512 fp32 O accumulator is exactly one SM's tensor memory, so
-//    splitting it over the pair (256 columns each) is what leaves room for
-//    the double-buffered score tiles.
-//  * Shared memory per CTA: Q 72 KB, two stages of (own tokens x 576 = 36 KB,
-//    all tokens x own latent = 32 KB), two P tiles of 8 KB. The second copy
-//    of latent columns is an L2 re-read; HBM sees each cached row once.
-//  * Warp roles: warp 0 issues TMA loads (both CTAs), warp 1 of CTA 0 issues
-//    the MMAs for the pair, warps 2-5 of both CTAs run the online softmax
-//    (fp32, exp2, lazy rescaling of O when the running max grows by more
-//    than 2^8) and the epilogue.
-//  * Work: the visible tiles of all token rows are concatenated and cut into
-//    equal contiguous ranges, one per cluster (persistent grid). A row whose
-//    tiles fall in one range is finished in place (bf16 o_lat, lse); a row cut
-//    by range boundaries leaves normalised fp32 partials that the combine
-//    kernel merges with a log-sum-exp.
+//  * All 128 heads of a token row share every cached row, so per 256-token
+//    tile S = Q K^T is a dense 128 x 256 x 576 contraction and O += P V a
+//    dense 128 x 512 x 256 one. Both run as tcgen05.mma.cta_group::2 on a
+//    pair of SMs (a 2-CTA cluster) with M = 128, N = 256: CTA r holds heads
+//    64r..64r+63 of Q, supplies tokens 128r..128r+127 of the tile to QK^T
+//    (B split by N = tokens) and latent columns [256j + 128r, +128) of every
+//    token to PV (B split by N = latent). Each MMA instruction then carries
+//    512K flop per SM, enough to keep the tensor pipe fed from one issuing
+//    thread (a tcgen05.mma takes ~25 ns to issue whatever its size).
+//  * The 128 x 512 fp32 accumulator O is one whole SM of tensor memory, so it
+//    is split over the pair: 256 columns per CTA, plus two 128-column score
+//    buffers = all 512 columns.
+//  * Shared memory per CTA: Q 72 KB resident per piece, P 32 KB, and one
+//    7-slot ring of 16 KB slabs consumed strictly in MMA order: the score
+//    slabs of tile i + 1 (per own block: 4 slabs of 2 column chunks + 1 of
+//    the last chunk), then the value slabs of tile i (per block: 2 slabs of
+//    128 latent columns). One ring for both operands keeps every slot in
+//    flight whichever product the tensor pipe is on. Latent columns are read
+//    twice from L2 (once per operand); HBM sees each cached row once.
+//  * Loads: 3-D / 4-D tensor maps view the cache as (64 columns, row, column
+//    chunk [, latent half]) with the chunk stride (128 B) smaller than the row
+//    stride, so one TMA instruction moves a whole 24-72 KB slab of a block
+//    straight into the chunk-major 128-byte-swizzled layout the MMAs read.
+//    (Many small 64 x 64 boxes cap TMA well below HBM bandwidth.)
+//  * QK^T is issued as N = 128 MMAs (64 tokens = one block per CTA) so each
+//    B operand is one contiguous block slab; PV uses N = 256 (latent).
+//  * Warp roles: warp 0 loads Q and fills the ring, warp 1 of CTA 0 issues
+//    the MMAs of the pair, warps 2-5 of both CTAs run the online softmax
+//    (fp32, exp2, O rescaled only when the running max grows by more than
+//    2^8) and the epilogue.
+//  * Work: the visible 256-token tiles of all token rows are concatenated and
+//    cut into equal contiguous ranges, one per cluster (persistent grid). A
+//    row whose tiles fall in one range is finished in place (bf16 o_lat,
+//    lse); a row cut by range boundaries leaves normalised fp32 partials
+//    that k_combine merges with a log-sum-exp.
+//  * Rows past a sequence's end: 64-row blocks wholly past it are loaded at
+//    an out-of-range coordinate (TMA zero fill); the one partially valid block
+//    has its value rows past the end zeroed in shared memory before its PV
+//    (scores there are masked to -inf, but 0 * NaN would still poison O).
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -35,40 +53,42 @@ namespace mla {
 namespace dec {
 
 constexpr int D = 576, DC = 512, DR = 64, HEADS = 128, HPC = 64;
-constexpr int TILE = 64, OWN = 32;
-constexpr int NS = 2;  // shared-memory stages
-constexpr int NB = 2;  // score / P buffers
-constexpr int NUM_THREADS = 192;
-constexpr int CHUNK_Q = HPC * 128;   // 64 rows x 128 B
-constexpr int CHUNK_KS = OWN * 128;  // 32 rows x 128 B
-constexpr int CHUNK_V = TILE * 128;  // 64 rows x 128 B
+constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CTA / per value chunk
+constexpr int NR = 7;                           // ring slots
+constexpr int NUM_THREADS = 192;                // 6 warps, see the role list in k_decode
+constexpr int CHUNK_Q = HPC * 128;   // 64 heads x 64 columns
+constexpr int ATOM_V = BLK * 128;    // 64 tokens x 64 columns (one 128-byte-swizzle atom column)
+constexpr int SLOT = 2 * ATOM_V;     // ring slot: 2 atoms
+constexpr int K_SLABS = 5;           // per own block: chunks {0,1} {2,3} {4,5} {6,7} {8}
+constexpr int LOADS_PER_TILE = 2 * K_SLABS + 4 * 2;  // score slabs (2 own blocks) + value slabs
+constexpr int CHUNK_P = HPC * 128;   // 64 heads x 64 tokens
 constexpr int Q_BYTES = 9 * CHUNK_Q;
-constexpr int KS_BYTES = 9 * CHUNK_KS;
-constexpr int V_BYTES = 4 * CHUNK_V;
-constexpr int P_BYTES = HPC * 128;
+constexpr int P_BYTES = 4 * CHUNK_P;
 constexpr int OFF_Q = 0;
-constexpr int OFF_KS = OFF_Q + Q_BYTES;
-constexpr int OFF_V = OFF_KS + NS * KS_BYTES;
-constexpr int OFF_P = OFF_V + NS * V_BYTES;
-constexpr int OFF_MISC = OFF_P + NB * P_BYTES;
-// misc: barriers then exchange arrays
-constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_KV_FULL = 2, BAR_KV_EMPTY = BAR_KV_FULL + NS,
-              BAR_S_FULL = BAR_KV_EMPTY + NS, BAR_S_FREE = BAR_S_FULL + NB, BAR_P_FULL = BAR_S_FREE + NB,
-              BAR_O_FULL = BAR_P_FULL + NB, BAR_O_FREE = BAR_O_FULL + NB, BAR_EXIT = BAR_O_FREE + 1,
-              NUM_BARS = BAR_EXIT + 1;
-constexpr int MISC_RED = 256;                 // float red[2][128]
-constexpr int MISC_REDL = MISC_RED + 1024;    // float redl[128]
-constexpr int MISC_INTS = MISC_REDL + 512;    // int scalars
+constexpr int OFF_P = OFF_Q + Q_BYTES;
+constexpr int OFF_R = OFF_P + P_BYTES;
+constexpr int OFF_MISC = OFF_R + NR * SLOT;
+constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_R_FULL = 2, BAR_R_EMPTY = BAR_R_FULL + NR,
+              BAR_V_LANDED = BAR_R_EMPTY + NR, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
+              BAR_S_FREE = BAR_S_FULL + 2,
+              BAR_P_FULL = BAR_S_FREE + 2, BAR_O_FULL = BAR_P_FULL + 1, BAR_O_FREE = BAR_O_FULL + 1,
+              BAR_EXIT = BAR_O_FREE + 1, NUM_BARS = BAR_EXIT + 1;
+constexpr int MISC_RED = 256;               // float red[2][128]
+constexpr int MISC_REDL = MISC_RED + 1024;  // float redl[128]
+constexpr int PF_TILES = 2;                 // L2 prefetch distance in tiles
+constexpr int MISC_INTS = MISC_REDL + 512;
 constexpr int MISC_BYTES = MISC_INTS + 64;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+static_assert(NUM_BARS * 8 <= MISC_RED, "barriers overlap the exchange arrays");
 static_assert(SMEM_BYTES <= 232448, "decode shared memory budget");
-constexpr int MAX_UNITS = V_BYTES / 4 - 1;  // plan scratch aliases the second V stage
-constexpr int S_COL = 256;                   // TMEM: O at [0,256), scores at [256, 256 + 32*NB)
-constexpr uint32_t IDESC_S = idesc_bf16(128, TILE, false, false);
+constexpr int MAX_UNITS = NR * SLOT / 4 - 1;  // plan scratch aliases the ring
+constexpr int S_COL = 256;                        // TMEM: O at [0,256), scores at [256 + 128 b, +128)
+constexpr uint32_t IDESC_S = idesc_bf16(128, 2 * BLK, false, false);  // N = one block per CTA
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
-constexpr float RESCALE_LOG2 = 8.f;  // rescale O only when the max grows by more than 2^8
+constexpr float RESCALE_LOG2 = 8.f;
 
 struct Params {
+  const uint8_t *cache;  // base of the cache rows (L2 prefetch addresses)
   const int32_t *seq_lens;
   const int32_t *block_table;
   int64_t max_len;
@@ -79,12 +99,12 @@ struct Params {
   float scale, scale_log2;
   __nv_bfloat16 *o_lat;
   float *lse;
-  float *part_o;     // [slots][128][512]
-  float *part_lse;   // [slots][128]
-  int32_t *plan;     // [0] = W, [1] = Qt, [2..] = tile offsets [BJ + 1]
+  float *part_o;    // [slots][128][512]
+  float *part_lse;  // [slots][128]
+  int32_t *plan;    // [0] = W, [1] = Qt, [2..] = tile offsets [BJ + 1]
 };
 
-// Tiles visible to unit bj (token row): 0 if its sequence length is invalid.
+// Tiles visible to unit bj (token row); -1 if its sequence length is invalid.
 __device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out) {
   const int b = bj / p.n_q, j = bj % p.n_q;
   const int L = p.seq_lens[b];
@@ -97,17 +117,16 @@ __device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out)
   return (vis + TILE - 1) / TILE;
 }
 
-// Physical cache row of the first token of tile `tile` of sequence b, or a
-// row past the end of the tensor map (TMA zero-fills it) if the block table
-// entry is out of range.
-__device__ __forceinline__ int32_t tile_row(const Params &p, int b, int tile) {
-  const int64_t pos = static_cast<int64_t>(tile) * TILE;
+// First cache row of the 64-row block at token `pos` of sequence b, or
+// p.cache_rows (out of range: the TMA load zero-fills) when the block lies
+// past `vis` or its block-table entry is invalid.
+__device__ __forceinline__ int32_t block_row(const Params &p, int b, int64_t pos, int vis) {
+  if (pos >= vis) return static_cast<int32_t>(p.cache_rows);
   if (!p.paged) return static_cast<int32_t>(static_cast<int64_t>(b) * p.max_len + pos);
-  const int64_t bi = pos / p.block_size;
-  const int32_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + bi];
+  const int32_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + pos / p.block_size];
   if (blk < 0 || blk >= p.num_blocks_i32) {
     dev_error(MLA_DEVERR_DATA);
-    return 0x7fffff00;
+    return static_cast<int32_t>(p.cache_rows);
   }
   return static_cast<int32_t>(static_cast<int64_t>(blk) * p.block_size + pos % p.block_size);
 }
@@ -148,6 +167,14 @@ struct PieceIter {
   }
 };
 
+// The value chunk of tile ti that needs zeroed rows (holds the last visible
+// token but not 64 visible tokens), or -1.
+__device__ __forceinline__ int partial_chunk(int vis, int ti) {
+  const int v = vis - ti * TILE;
+  if (v >= TILE || (v % BLK) == 0) return -1;
+  return v / BLK;
+}
+
 __device__ __forceinline__ void arrive_leader(uint32_t bar_local, uint32_t rank) {
   if (rank == 0)
     mbar_arrive(bar_local);
@@ -156,8 +183,9 @@ __device__ __forceinline__ void arrive_leader(uint32_t bar_local, uint32_t rank)
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
-    k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
-             const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k2,
+             const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_v0,
+             const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -178,33 +206,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
     mbar_init(bar(BAR_Q_EMPTY), 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(bar(BAR_KV_FULL + s), 1);
-      mbar_init(bar(BAR_KV_EMPTY + s), 1);
+    for (int s = 0; s < NR; ++s) {
+      mbar_init(bar(BAR_R_FULL + s), 1);
+      mbar_init(bar(BAR_R_EMPTY + s), 1);
     }
-    for (int b = 0; b < NB; ++b) {
+    mbar_init(bar(BAR_V_LANDED), 1);
+    mbar_init(bar(BAR_ZERO_DONE), 8);
+    for (int b = 0; b < 2; ++b) {
       mbar_init(bar(BAR_S_FULL + b), 1);
       mbar_init(bar(BAR_S_FREE + b), 8);
-      mbar_init(bar(BAR_P_FULL + b), 8);
-      mbar_init(bar(BAR_O_FULL + b), 1);
     }
+    mbar_init(bar(BAR_P_FULL), 8);
+    mbar_init(bar(BAR_O_FULL), 1);
     mbar_init(bar(BAR_O_FREE), 8);
     mbar_init(bar(BAR_EXIT), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  const CUtensorMap *tm_v = rank == 0 ? &tm_v0 : &tm_v1;  // value slabs: this CTA's latent columns
   if (warp == 0) {
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_ks);
-    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_k2);
+    tma_prefetch_desc(&tm_k1);
+    tma_prefetch_desc(tm_v);
   }
-  if (warp == 1) {
-    tmem_alloc<2>(smem_u32(tmem_slot), 512);
-  }
+  if (warp == 1) tmem_alloc<2>(smem_u32(tmem_slot), 512);
 
   // ---- plan: tiles per unit, prefix sums, this cluster's first unit ----
   const int BJ = p.B * p.n_q;
-  int *scratch = reinterpret_cast<int *>(smem + OFF_V + V_BYTES);
+  int *scratch = reinterpret_cast<int *>(smem + OFF_R);
   for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
     int vis;
     int nt = unit_tiles(p, u, &vis);
@@ -216,7 +246,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   }
   __syncthreads();
   {
-    // each thread scans a contiguous segment; block scan of the segment sums
     const int per = (BJ + NUM_THREADS - 1) / NUM_THREADS;
     const int lo = threadIdx.x * per, hi = min(BJ, lo + per);
     int sum = 0;
@@ -232,7 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     __syncthreads();
     int base = 0;
     for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    int run = base + incl - sum;  // exclusive prefix of this segment
+    int run = base + incl - sum;
     for (int u = lo; u < hi; ++u) {
       const int nt = scratch[u];
       scratch[u] = run;
@@ -243,7 +272,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       for (int w = 0; w < NUM_THREADS / 32; ++w) W += warp_tot[w];
       plan_s[0] = W;
       plan_s[1] = max(1, (W + nclusters - 1) / nclusters);
-      plan_s[2] = BJ;  // bj_first (none yet)
+      plan_s[2] = BJ;
       plan_s[3] = W;
     }
     __syncthreads();
@@ -281,199 +310,275 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   it0.k = cluster;
 
   if (warp == 0) {
-    // ------------------------------------------------------------- producer
+    // --------------------------------------------------------- ring producer
+    // Load order = MMA consumption order: per piece Q, then score slabs of
+    // tile 0, and for every later tile its score slabs followed by the value
+    // slabs of the tile before it; the last tile's value slabs close the
+    // piece. Block rows of a tile are read one tile before they are needed.
     if (lane == 0) {
       const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
-      uint32_t kv_full[NS];
-      for (int s = 0; s < NS; ++s)
-        kv_full[s] = rank == 0 ? bar(BAR_KV_FULL + s) : mapa_shared(bar(BAR_KV_FULL + s), 0);
       PieceIter it = it0;
       Piece pc;
-      int gi = 0, npc = 0;
+      int g = 0, npc = 0;
       bool ok = true;
+      auto slot_for_load = [&](uint32_t bytes) -> int {  // wait for a free slot, arm its barrier
+        const int s = g % NR;
+        if (g >= NR && !mbar_wait(bar(BAR_R_EMPTY + s), ((g / NR) - 1) & 1, abort_flag)) return -1;
+        if (rank == 0) mbar_arrive_expect_tx(bar(BAR_R_FULL + s), 2 * bytes);
+        return s;
+      };
+      auto full_of = [&](int s) { return rank == 0 ? bar(BAR_R_FULL + s) : mapa_shared(bar(BAR_R_FULL + s), 0); };
+      auto load_k = [&](const int32_t *own) -> bool {  // score slabs of one tile (own blocks)
+        for (int kb = 0; kb < 2; ++kb)
+          for (int m = 0; m < K_SLABS; ++m) {
+            const bool last = m == K_SLABS - 1;
+            const int s = slot_for_load(last ? ATOM_V : SLOT);
+            if (s < 0) return false;
+            tma_load_3d_pair(sbase + OFF_R + s * SLOT, last ? &tm_k1 : &tm_k2, 0, own[kb], 2 * m, full_of(s));
+            ++g;
+          }
+        return true;
+      };
+      auto load_v = [&](const int32_t *rows) -> bool {  // value slabs of one tile (all 4 blocks)
+        for (int v = 0; v < 4; ++v)
+          for (int j = 0; j < 2; ++j) {
+            const int s = slot_for_load(SLOT);
+            if (s < 0) return false;
+            tma_load_4d_pair(sbase + OFF_R + s * SLOT, tm_v, 0, rows[v], 0, j, full_of(s));
+            ++g;
+          }
+        return true;
+      };
       while (ok && it.next(p, pc)) {
+        const int b = pc.bj / p.n_q;
+        auto rows_of = [&](int ti, int32_t *r4) {
+          for (int v = 0; v < 4; ++v) r4[v] = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * v, pc.vis);
+        };
+        int32_t cur[4], prev[4], nxt[4];
+        rows_of(pc.t_begin, cur);
         if (npc > 0 && !mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         if (rank == 0) mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * Q_BYTES);
-        for (int c = 0; c < 9; ++c)
-          tma_load_2d_pair(sbase + OFF_Q + c * CHUNK_Q, &tm_q, 64 * c, pc.bj * HEADS + HPC * rank, q_full);
-        const int b = pc.bj / p.n_q;
-        for (int ti = pc.t_begin; ti < pc.t_end; ++ti, ++gi) {
-          const int s = gi % NS;
-          if (gi >= NS && !mbar_wait(bar(BAR_KV_EMPTY + s), ((gi / NS) - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
+        tma_load_3d_pair(sbase + OFF_Q, &tm_q, 0, pc.bj * HEADS + HPC * rank, 0, q_full);
+        for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti) {
+          if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
+          const int32_t own[2] = {cur[2 * rank], cur[2 * rank + 1]};
+          if (!load_k(own)) { ok = false; break; }
+          if (ti > pc.t_begin && !load_v(prev)) { ok = false; break; }
+          for (int v = 0; v < 4; ++v) {
+            prev[v] = cur[v];
+            cur[v] = nxt[v];
           }
-          const int32_t row0 = tile_row(p, b, ti);
-          if (rank == 0) mbar_arrive_expect_tx(bar(BAR_KV_FULL + s), 2 * (KS_BYTES + V_BYTES));
-          const uint32_t ks = sbase + OFF_KS + s * KS_BYTES;
-          const uint32_t vv = sbase + OFF_V + s * V_BYTES;
-          for (int c = 0; c < 9; ++c) tma_load_2d_pair(ks + c * CHUNK_KS, &tm_ks, 64 * c, row0 + OWN * rank, kv_full[s]);
-          for (int c = 0; c < 4; ++c)
-            tma_load_2d_pair(vv + c * CHUNK_V, &tm_v, 256 * (c >> 1) + 128 * rank + 64 * (c & 1), row0, kv_full[s]);
         }
+        if (!ok || !load_v(prev)) { ok = false; break; }
         ++npc;
       }
       // drain: every commit aimed at this CTA's empty barriers has landed
       if (ok && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
-      for (int g = gi - NS; ok && g < gi; ++g)
-        if (g >= 0) mbar_wait(bar(BAR_KV_EMPTY + g % NS), (g / NS) & 1, abort_flag);
+      for (int q = g - NR; ok && q < g; ++q)
+        if (q >= 0) mbar_wait(bar(BAR_R_EMPTY + q % NR), (q / NR) & 1, abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0) {
       PieceIter it = it0;
-      Piece pc;
-      int gi = 0, npc = 0;
+      Piece pc{};
+      int gi = 0, g = 0, gz = 0, npc = 0;
       bool ok = true;
-      auto issue_pv = [&](int g, bool first) -> bool {
-        const int b = g % NB, s = g % NS;
-        if (!mbar_wait(bar(BAR_P_FULL + b), (g / NB) & 1, abort_flag)) return false;
-        if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+      auto take = [&]() -> int {  // next ring slot in consumption order, once it has landed
+        const int s = g % NR;
+        if (!mbar_wait(bar(BAR_R_FULL + s), (g / NR) & 1, abort_flag)) return -1;
         tc_fence_after();
-        const uint32_t pbase = sbase + OFF_P + b * P_BYTES;
-        const uint32_t vbase = sbase + OFF_V + s * V_BYTES;
+        return s;
+      };
+      auto release = [&](int s) {
+        tc_commit_pair(bar(BAR_R_EMPTY + s), 0x3);
+        ++g;
+      };
+      // PV of global tile gt (tile ti of the current piece)
+      auto issue_pv = [&](int gt, int ti, bool first) -> bool {
+        const int zc = partial_chunk(pc.vis, ti);
+        for (int v = 0; v < 4; ++v)
+          for (int j = 0; j < 2; ++j) {
+            const int s = take();
+            if (s < 0) return false;
+            if (v == 0 && j == 0) {
+              if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
+              if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+            }
+            if (v == zc) {  // both CTAs zero the rows past the end of this slab first
+              mbar_arrive(bar(BAR_V_LANDED));
+              mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
+              if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
+              ++gz;
+              tc_fence_after();
+            }
+            const uint32_t pa = sbase + OFF_P + v * CHUNK_P;
+            const uint32_t vb = sbase + OFF_R + s * SLOT;
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int kk = 0; kk < TILE / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(pbase + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(vbase + (2 * j) * CHUNK_V + kk * 2048, CHUNK_V, 1024);
-            tc_mma<2>(tmem + 128 * j, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma<2>(tmem + 128 * j, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(vb + kk * 2048, ATOM_V, 1024),
+                        IDESC_PV, (first && v == 0 && kk == 0) ? 0u : 1u);
+            release(s);
           }
-        tc_commit_pair(bar(BAR_O_FULL + b), 0x3);
-        tc_commit_pair(bar(BAR_KV_EMPTY + s), 0x3);
+        tc_commit_pair(bar(BAR_O_FULL), 0x3);
         return true;
       };
       while (ok && it.next(p, pc)) {
-        if (!mbar_wait(bar(BAR_Q_FULL), npc & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(bar(BAR_Q_FULL), npc & 1, abort_flag)) break;
         const int n = pc.t_end - pc.t_begin;
-        for (int i = 0; i < n; ++i, ++gi) {
-          const int s = gi % NS, b = gi % NB;
-          if (!mbar_wait(bar(BAR_KV_FULL + s), (gi / NS) & 1, abort_flag)) { ok = false; break; }
-          if (gi >= NB && !mbar_wait(bar(BAR_S_FREE + b), ((gi / NB) - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ks = sbase + OFF_KS + s * KS_BYTES;
+        for (int i = 0; i < n && ok; ++i, ++gi) {
+          const int b = gi & 1;
+          if (gi >= 2 && !mbar_wait(bar(BAR_S_FREE + b), ((gi >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          for (int kb = 0; kb < 2 && ok; ++kb)
+            for (int m = 0; m < K_SLABS; ++m) {
+              const int s = take();
+              if (s < 0) { ok = false; break; }
+              const uint32_t slab = sbase + OFF_R + s * SLOT;
+              const int nch = m == K_SLABS - 1 ? 1 : 2;
+              for (int c = 0; c < nch; ++c)
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const int c = k >> 2, kk = k & 3;
-            const uint64_t ad = sdesc_sw128(sbase + OFF_Q + c * CHUNK_Q + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(ks + c * CHUNK_KS + kk * 32, 16, 1024);
-            tc_mma<2>(tmem + S_COL + 32 * b, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
-          }
+                for (int kk = 0; kk < 4; ++kk)
+                  tc_mma<2>(tmem + S_COL + 128 * b + 64 * kb,
+                            sdesc_sw128(sbase + OFF_Q + (2 * m + c) * CHUNK_Q + kk * 32, 16, 1024),
+                            sdesc_sw128(slab + c * ATOM_V + kk * 32, 16, 1024), IDESC_S,
+                            (m > 0 || c > 0 || kk > 0) ? 1u : 0u);
+              release(s);
+            }
+          if (!ok) break;
           tc_commit_pair(bar(BAR_S_FULL + b), 0x3);
           if (i == n - 1) tc_commit_pair(bar(BAR_Q_EMPTY), 0x3);
-          if (i > 0 && !issue_pv(gi - 1, i == 1)) { ok = false; break; }
+          if (i > 0 && !issue_pv(gi - 1, pc.t_begin + i - 1, i == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!issue_pv(gi - 1, n == 1)) { ok = false; break; }
+        if (!issue_pv(gi - 1, pc.t_end - 1, n == 1)) break;
         ++npc;
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------- softmax + epilogue
-    const int sp = warp & 3;               // TMEM sub-partition of this warp
-    const int L = 32 * sp + lane;          // TMEM lane
-    const int row = L & 63, half = L >> 6;  // head within CTA, token / latent half
+    // A failed (timed-out) wait does not break these loops: every softmax
+    // warp keeps the same sequence of named-barrier syncs and runs to the
+    // end on whatever data is there; the device error word reports it.
+    const int sp = warp & 3;                // TMEM sub-partition of this warp
+    const int L = 32 * sp + lane;           // TMEM lane
+    const int row = L & 63, half = L >> 6;  // head within CTA; token half / latent half
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
     const float c2 = p.scale_log2;
     PieceIter it = it0;
     Piece pc;
-    int gi = 0;
-    // A failed (timed-out) wait does not break these loops: every softmax
-    // warp keeps the same sequence of named-barrier syncs and runs to the
-    // end on whatever data is there; the device error word reports it.
+    int gi = 0, gz = 0, gbase = 0;  // gbase: ring loads before this piece
     while (it.next(p, pc)) {
       const int n = pc.t_end - pc.t_begin;
       float m_ref = -INFINITY, lsum = 0.f;
       for (int i = 0; i < n; ++i, ++gi) {
-        const int b = gi % NB, ti = pc.t_begin + i;
-        mbar_wait_warp(bar(BAR_S_FULL + b), (gi / NB) & 1, abort_flag);
+        const int b = gi & 1, ti = pc.t_begin + i;
+        const int vis_t = pc.vis - ti * TILE;  // visible tokens of this tile
+        const int tok0 = OWN * half;            // this thread's first token within the tile
+        mbar_wait_warp(bar(BAR_S_FULL + b), (gi >> 1) & 1, abort_flag);
         tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld32(lane_addr + S_COL + 32 * b, sr);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_leader(bar(BAR_S_FREE + b), rank);
-        float sv[32];
-        const int tok0 = ti * TILE + OWN * half;
+        const uint32_t s_addr = lane_addr + S_COL + 128 * b;
+        // pass 1: row max over this thread's 128 tokens, then with the partner lane
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t sr[32];
+          tmem_ld32(s_addr + 32 * q4, sr);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c] = (tok0 + c < pc.vis) ? __uint_as_float(sr[c]) : -INFINITY;
-        float mx = sv[0];
-#pragma unroll
-        for (int c = 1; c < 32; ++c) mx = fmaxf(mx, sv[c]);
+          for (int c = 0; c < 32; ++c)
+            if (tok0 + 32 * q4 + c < vis_t) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        }
         red[(gi & 1) * 128 + L] = mx;
         named_bar_sync(1, 128);
         mx = fmaxf(mx, red[(gi & 1) * 128 + (L ^ 64)]);
+        bool rescale = false;
+        float alpha = 1.f;
         if (i == 0) {
           m_ref = mx;
         } else {
           const bool need = (mx - m_ref) * c2 > RESCALE_LOG2;
-          if (__any_sync(0xffffffffu, need)) {
-            const float m_new = need ? mx : m_ref;
-            const float alpha = exp2f((m_ref - m_new) * c2);
-            const int gp = gi - 1;  // wait until PV of the previous tile has landed in O
-            mbar_wait_warp(bar(BAR_O_FULL + gp % NB), (gp / NB) & 1, abort_flag);
-            tc_fence_after();
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const uint32_t a = lane_addr + 128 * (q4 >> 2) + 32 * (q4 & 3);
-              uint32_t o[32];
-              tmem_ld32(a, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              tmem_st32(a, o);
-            }
-            tmem_wait_st();
-            lsum *= alpha;
-            m_ref = m_new;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx((m_ref - mx) * c2);
+            m_ref = mx;
           }
         }
+        // pass 2: p = exp2((s - m) * scale * log2 e), packed to bf16 in registers
         const float mo = m_ref * c2;
-        uint32_t pk[16];
+        uint32_t pk[64];
         float ps = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = exp2f(fmaf(sv[2 * c], c2, -mo));
-          const float p1 = exp2f(fmaf(sv[2 * c + 1], c2, -mo));
-          ps += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        lsum += ps;
-        // the P buffer is free once the PV of two tiles ago has completed
-        if (gi >= NB) mbar_wait_warp(bar(BAR_O_FULL + b), ((gi - NB) / NB) & 1, abort_flag);
-        uint8_t *pb = smem + OFF_P + b * P_BYTES + row * 128;
-#pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int chunk = 4 * half + q4;
-          *reinterpret_cast<uint4 *>(pb + ((chunk ^ (row & 7)) << 4)) =
-              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
-        // last, partial tile: zero the value rows past the end (they may hold
-        // anything, and 0 * NaN would poison O)
-        const int valid = pc.vis - ti * TILE;
-        if (valid < TILE) {
-          uint8_t *vb = smem + OFF_V + (gi % NS) * V_BYTES;
-          const int nrow = TILE - valid;
-          for (int e = L; e < nrow * 4 * 8; e += 128) {
-            const int r = valid + e / 32, c = (e >> 3) & 3, w16 = e & 7;
-            *reinterpret_cast<uint4 *>(vb + c * CHUNK_V + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
+          uint32_t sr[32];
+          tmem_ld32(s_addr + 32 * q4, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int t = tok0 + 32 * q4 + 2 * c;
+            const float p0 = t < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c]), c2, -mo)) : 0.f;
+            const float p1 = t + 1 < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), c2, -mo)) : 0.f;
+            ps += p0 + p1;
+            pk[16 * q4 + c] = pack_bf16x2(p0, p1);
           }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader(bar(BAR_S_FREE + b), rank);
+        // the single P buffer and O are free once the previous tile's PV is done
+        if (gi > 0) mbar_wait_warp(bar(BAR_O_FULL), (gi - 1) & 1, abort_flag);
+        tc_fence_after();
+        if (rescale) {
+#pragma unroll 1
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const uint32_t a = lane_addr + 128 * (q4 >> 2) + 32 * (q4 & 3);
+            uint32_t o[32];
+            tmem_ld32(a, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(a, o);
+          }
+          tmem_wait_st();
+        }
+        lsum = lsum * alpha + ps;
+        // P: row `row`, tokens tok0 .. tok0 + 127 -> chunks 2*half, 2*half + 1 (SW128, K-major)
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int chunk = 2 * half + (u >> 3), w16 = u & 7;
+          uint8_t *dst = smem + OFF_P + chunk * CHUNK_P + row * 128 + ((w16 ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) arrive_leader(bar(BAR_P_FULL + b), rank);
+        if (lane == 0) arrive_leader(bar(BAR_P_FULL), rank);
+        // partial block of the last tile: zero value rows past the end in its
+        // two slabs (the MMA thread signals each one as it reaches it)
+        const int zc = partial_chunk(pc.vis, ti);
+        if (zc >= 0) {
+          // ring index of this tile's value slabs (see the producer's order)
+          const int kt = i, nt_p = n;
+          const int gv = gbase + K_SLABS * 2 * min(kt + 2, nt_p) + 8 * kt + 2 * zc;
+          const int valid = vis_t - BLK * zc;
+          const int nrow = BLK - valid;
+          for (int j = 0; j < 2; ++j) {
+            mbar_wait_warp(bar(BAR_V_LANDED), gz & 1, abort_flag);
+            ++gz;
+            uint8_t *vb = smem + OFF_R + ((gv + j) % NR) * SLOT;
+            for (int e = L; e < nrow * 2 * 8; e += 128) {
+              const int r = valid + e / 16, a = (e >> 3) & 1, w16 = e & 7;
+              *reinterpret_cast<uint4 *>(vb + a * ATOM_V + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) arrive_leader(bar(BAR_ZERO_DONE), rank);
+          }
+        }
       }
       // ---------------------------------------------------------- epilogue
-      const int gl = gi - 1;
-      mbar_wait_warp(bar(BAR_O_FULL + gl % NB), (gl / NB) & 1, abort_flag);
+      mbar_wait_warp(bar(BAR_O_FULL), (gi - 1) & 1, abort_flag);
       tc_fence_after();
       redl[L] = lsum;
       named_bar_sync(1, 128);
@@ -516,6 +621,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(bar(BAR_O_FREE), rank);
+      gbase += LOADS_PER_TILE * n;
     }
   }
 

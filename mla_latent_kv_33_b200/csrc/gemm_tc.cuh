@@ -21,6 +21,14 @@ namespace gemm {
 constexpr int BM = 128, BK = 64, NUM_THREADS = 192;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 
+// Epilogue of one GEMM launch.
+enum Epi : int {
+  EPI_PARTIAL = 0,  // fp32 partial sums: out[batch][split][n][m]
+  EPI_BF16 = 1,     // bf16 dst[batch * e_bs + n * e_ns + m]
+  EPI_UQ = 2,       // rows < e_split: bf16 q_C at dst[n * e_split + m]; rows above: q_R rotated
+                    // by RoPE at positions[n], stored at q[n][h][d_c + i] (m - e_split = h * d_r + i)
+};
+
 struct Params {
   int m_total;       // rows of D per batch
   int m_split;       // rows [m_split, m_total) come from the second A map
@@ -33,13 +41,21 @@ struct Params {
   int a_batch_rows;  // A row offset per batch (K-major: m rows; MN-major: k rows)
   int b_batch_cols;  // B column (k) offset per batch
   int stages;
-  float *out;        // [batch][split][n_total][m_total]
+  float *out;        // EPI_PARTIAL: [batch][split][n_total][m_total]
+  int epi;
+  __nv_bfloat16 *dst;  // EPI_BF16 / EPI_UQ (q_C)
+  int64_t e_bs, e_ns;  // EPI_BF16 strides
+  int e_split;         // EPI_UQ: first q_R row
+  __nv_bfloat16 *q;    // EPI_UQ: q[T][n_h][d_c + d_r]
+  int n_h, d_c, d_r;
+  double rope_base;
+  const int32_t *positions;
 };
 
 __host__ __device__ constexpr int b_stage_bytes(int n_tile) { return n_tile * BK * 2; }
 
 // One CTA: M tile blockIdx.x, N tile blockIdx.y, (batch, split) blockIdx.z.
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 2)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
            const __grid_constant__ CUtensorMap tm_b, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -126,18 +142,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_wait_warp(done, 0, abort_flag);
     tc_fence_after();
     const int m = m0 + row;
-    float *out = p.out + (static_cast<int64_t>(batch) * p.splits + split) * p.n_total * p.m_total;
     const int n_base = n_tile * p.n_tile;
+    float *out = p.out + (static_cast<int64_t>(batch) * p.splits + split) * p.n_total * p.m_total;
+    const bool rope_tile = p.epi == EPI_UQ && m0 >= p.e_split;  // whole M tiles are q_C or q_R
     for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
       uint32_t v[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + c0, v);
       tmem_wait_ld();
-      if (m < p.m_total) {
+      if (nkb == 0) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = 0u;
+      }
+      if (p.epi == EPI_PARTIAL) {
+        if (m < p.m_total) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int n = n_base + c0 + c;
+            if (c0 + c < p.n_tile && n < p.n_total) out[static_cast<int64_t>(n) * p.m_total + m] = __uint_as_float(v[c]);
+          }
+        }
+      } else if (p.epi == EPI_BF16) {
+        if (m < p.m_total) {
+          __nv_bfloat16 *d = p.dst + batch * p.e_bs + m;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int n = n_base + c0 + c;
+            if (c0 + c < p.n_tile && n < p.n_total) d[n * p.e_ns] = __float2bfloat16_rn(__uint_as_float(v[c]));
+          }
+        }
+      } else if (!rope_tile) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int n = n_base + c0 + c;
           if (c0 + c < p.n_tile && n < p.n_total)
-            out[static_cast<int64_t>(n) * p.m_total + m] = nkb > 0 ? __uint_as_float(v[c]) : 0.f;
+            p.dst[static_cast<int64_t>(n) * p.e_split + m] = __float2bfloat16_rn(__uint_as_float(v[c]));
+        }
+      } else {
+        // q_R rows: lanes (2k, 2k+1) hold the RoPE pair (x[2i], x[2i+1])
+        const int r = m - p.e_split, h = r / p.d_r, i = r % p.d_r;
+        const bool odd = (i & 1) != 0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int n = n_base + c0 + c;
+          const float mine = __uint_as_float(v[c]);
+          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          if (c0 + c < p.n_tile && n < p.n_total) {
+            float x0 = odd ? other : mine, x1 = odd ? mine : other;
+            rope_pair(x0, x1, i >> 1, p.d_r, p.positions[n], p.rope_base);
+            p.q[(static_cast<int64_t>(n) * p.n_h + h) * (p.d_c + p.d_r) + p.d_c + i] = __float2bfloat16_rn(odd ? x1 : x0);
+          }
         }
       }
     }
@@ -149,33 +202,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ---------------------------------------------------------- finalizers ----
 
-__device__ __forceinline__ float sum_splits(const float *part, int splits, int64_t stride, int64_t idx) {
-  float acc = 0.f;
-  for (int s = 0; s < splits; ++s) acc += part[s * stride + idx];
-  return acc;
+__device__ __forceinline__ float2 sum_splits2(const float *part, int splits, int64_t stride, int64_t idx) {
+  float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+  int s = 0;
+  for (; s + 4 <= splits; s += 4) {
+    const float2 v0 = *reinterpret_cast<const float2 *>(part + (s + 0) * stride + idx);
+    const float2 v1 = *reinterpret_cast<const float2 *>(part + (s + 1) * stride + idx);
+    const float2 v2 = *reinterpret_cast<const float2 *>(part + (s + 2) * stride + idx);
+    const float2 v3 = *reinterpret_cast<const float2 *>(part + (s + 3) * stride + idx);
+    a.x += v0.x + v1.x;
+    a.y += v0.y + v1.y;
+    b.x += v2.x + v3.x;
+    b.y += v2.y + v3.y;
+  }
+  for (; s < splits; ++s) {
+    const float2 v = *reinterpret_cast<const float2 *>(part + s * stride + idx);
+    a.x += v.x;
+    a.y += v.y;
+  }
+  return make_float2(a.x + b.x, a.y + b.y);
 }
 
 // rows [T][576] = sum of splits; RoPE on [512, 576); bf16; store at the
-// cache row of (seq_idx[t], positions[t]). One block of 288 threads per
-// token, one thread per element pair.
+// cache row of (seq_idx[t], positions[t]). grid (ceil(D / 256), T), one
+// thread per element pair.
 __global__ void k_fin_append(const float *part, int splits, int T, int d_c, int d_r, double rope_base,
                              const int32_t *seq_idx, const int32_t *positions, CacheView cache) {
-  const int t = blockIdx.x;
+  const int t = blockIdx.y;
   const int D = d_c + d_r;
+  const int e = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (e >= D) return;
   const int64_t stride = static_cast<int64_t>(T) * D;
   const int pos = positions[t];
   const int64_t row = cache_row(cache, seq_idx[t], pos);
   if (row < 0) {
-    if (threadIdx.x == 0) dev_error(MLA_DEVERR_DATA);
+    if (e == 0) dev_error(MLA_DEVERR_DATA);
     return;
   }
   __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(cache.data) + row * D;
-  for (int e = 2 * threadIdx.x; e < D; e += 2 * blockDim.x) {
-    float x0 = sum_splits(part, splits, stride, static_cast<int64_t>(t) * D + e);
-    float x1 = sum_splits(part, splits, stride, static_cast<int64_t>(t) * D + e + 1);
-    if (e >= d_c) rope_pair(x0, x1, (e - d_c) / 2, d_r, pos, rope_base);
-    *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(x0, x1);
-  }
+  const float2 x = sum_splits2(part, splits, stride, static_cast<int64_t>(t) * D + e);
+  float x0 = x.x, x1 = x.y;
+  if (e >= d_c) rope_pair(x0, x1, (e - d_c) / 2, d_r, pos, rope_base);
+  *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(x0, x1);
 }
 
 // dst[t][n] (bf16, row pitch ld) = sum of splits of part[.][t][n], n < N.
@@ -184,55 +252,16 @@ __global__ void k_fin_store(const float *part, int splits, int T, int N, __nv_bf
   for (int64_t i = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); i < stride;
        i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t t = i / N, n = i % N;
-    const float x0 = sum_splits(part, splits, stride, i), x1 = sum_splits(part, splits, stride, i + 1);
-    *reinterpret_cast<uint32_t *>(dst + t * ld + n) = pack_bf16x2(x0, x1);
+    const float2 x = sum_splits2(part, splits, stride, i);
+    *reinterpret_cast<uint32_t *>(dst + t * ld + n) = pack_bf16x2(x.x, x.y);
   }
 }
 
-// [W_UQ; W_QR] c_Q partials: rows < n_h*d_h are q_C (bf16 [T][n_h*d_h]);
-// rows above are q_R before RoPE: rotate and store into q[t][h][d_c + r].
-__global__ void k_fin_uq(const float *part, int splits, int T, int n_h, int d_h, int d_c, int d_r,
-                         double rope_base, const int32_t *positions, __nv_bfloat16 *qc, __nv_bfloat16 *q) {
-  const int M = n_h * (d_h + d_r);
-  const int64_t stride = static_cast<int64_t>(T) * M;
-  const int t = blockIdx.y;
-  const int pos = positions[t];
-  for (int e = 2 * (blockIdx.x * blockDim.x + threadIdx.x); e < M; e += 2 * gridDim.x * blockDim.x) {
-    float x0 = sum_splits(part, splits, stride, static_cast<int64_t>(t) * M + e);
-    float x1 = sum_splits(part, splits, stride, static_cast<int64_t>(t) * M + e + 1);
-    if (e < n_h * d_h) {
-      *reinterpret_cast<uint32_t *>(qc + static_cast<int64_t>(t) * n_h * d_h + e) = pack_bf16x2(x0, x1);
-    } else {
-      const int r = e - n_h * d_h, h = r / d_r, i = r % d_r;
-      rope_pair(x0, x1, i / 2, d_r, pos, rope_base);
-      *reinterpret_cast<uint32_t *>(q + (static_cast<int64_t>(t) * n_h + h) * (d_c + d_r) + d_c + i) =
-          pack_bf16x2(x0, x1);
-    }
-  }
-}
-
-// Per-head partials part[h][split][t][m] (m < M) -> bf16 dst[t][h][m] with
-// head pitch hp and token pitch tp.
-__global__ void k_fin_heads(const float *part, int splits, int T, int M, int n_h, __nv_bfloat16 *dst,
-                            int64_t tp, int64_t hp) {
-  const int h = blockIdx.y;
-  const int64_t stride = static_cast<int64_t>(T) * M;
-  const float *ph = part + static_cast<int64_t>(h) * splits * stride;
-  for (int64_t i = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); i < stride;
-       i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / M, m = i % M;
-    const float x0 = sum_splits(ph, splits, stride, i), x1 = sum_splits(ph, splits, stride, i + 1);
-    *reinterpret_cast<uint32_t *>(dst + t * tp + h * hp + m) = pack_bf16x2(x0, x1);
-  }
-  (void)n_h;
-}
-
-// Split-K choice: enough CTAs to cover the GPU about twice, at least 2 K
-// blocks per split where K allows.
+// Split-K choice: about one CTA per SM, at least 4 K blocks per split.
 inline int choose_splits(int tiles, int k_blocks, int sms) {
-  int s = (2 * sms + tiles - 1) / tiles;
+  int s = (sms + tiles - 1) / tiles;
   s = s < 1 ? 1 : s;
-  const int max_s = k_blocks >= 4 ? k_blocks / 2 : k_blocks;
+  const int max_s = k_blocks >= 8 ? k_blocks / 4 : 1;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   // equalise: every split gets ceil(k_blocks / s) blocks
@@ -245,10 +274,11 @@ inline int n_tile_for(int T) {
   return n < 16 ? 16 : n;
 }
 
+// Pipeline depth: fit two CTAs per SM where the N tile allows (~100 KB each).
 inline int stages_for(int n_tile) {
-  const int budget = 200 * 1024;
+  const int budget = 100 * 1024;
   int s = budget / (A_STAGE + b_stage_bytes(n_tile));
-  return s > 8 ? 8 : (s < 2 ? 2 : s);
+  return s > 8 ? 8 : (s < 3 ? 3 : s);
 }
 
 inline size_t smem_for(int n_tile, int stages) {

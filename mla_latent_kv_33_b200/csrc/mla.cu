@@ -226,25 +226,36 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [outer][inner] array with row pitch
-// `pitch_bytes`, box [box_outer][box_inner], 128-byte swizzle. Encoded maps
-// are kept in a small per-thread cache keyed by all of their arguments.
+// bf16 tensor map of rank 2..4 with 128-byte swizzle: dims[0] is the
+// contiguous dimension, strides[i] is the byte stride of dims[i + 1]. Encoded
+// maps are kept in a small per-thread cache keyed by all of their arguments.
 struct TmapKey {
   const void *base;
-  uint64_t inner, outer, pitch;
-  uint32_t bi, bo;
+  int rank;
+  uint64_t dims[4], strides[3];
+  uint32_t box[4];
   bool operator==(const TmapKey &o) const {
-    return base == o.base && inner == o.inner && outer == o.outer && pitch == o.pitch && bi == o.bi && bo == o.bo;
+    if (base != o.base || rank != o.rank) return false;
+    for (int i = 0; i < rank; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i] || (i + 1 < rank && strides[i] != o.strides[i])) return false;
+    return true;
   }
 };
 
-mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
-                          uint32_t box_inner, uint32_t box_outer, const char *what) {
+mla_status make_tmap_nd(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides,
+                        const uint32_t *box, const char *what) {
   constexpr int CAP = 64;
   thread_local TmapKey keys[CAP];
   thread_local CUtensorMap maps[CAP];
   thread_local int used = 0, next = 0;
-  const TmapKey key{base, inner, outer, pitch_bytes, box_inner, box_outer};
+  TmapKey key{};
+  key.base = base;
+  key.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides[i];
+  }
   for (int i = 0; i < used; ++i)
     if (keys[i] == key) {
       *m = maps[i];
@@ -252,19 +263,30 @@ mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint
     }
   auto fn = encode_fn();
   if (fn == nullptr) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {pitch_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t d[4], st[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, st,
+                  bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "tensor map for %s: CUresult %d", what, static_cast<int>(r));
   keys[next] = key;
   maps[next] = *m;
   next = (next + 1) % CAP;
   if (used < CAP) ++used;
   return MLA_OK;
+}
+
+// 2-D map over a row-major [outer][inner] array with row pitch `pitch_bytes`.
+mla_status make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
+                          uint32_t box_inner, uint32_t box_outer, const char *what) {
+  const uint64_t dims[2] = {inner, outer}, strides[1] = {pitch_bytes};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return make_tmap_nd(m, base, 2, dims, strides, box, what);
 }
 
 // ------------------------------------------------ tensor-core projections --
@@ -275,7 +297,8 @@ struct GemmShape {
   int m_total, m_tiles, n_tile, n_tiles, k_blocks, splits, batches;
 };
 
-GemmShape gemm_shape(int m_total, int T, int K, int batches) {
+// split_k = false: one CTA per output tile, epilogue fused into the GEMM.
+GemmShape gemm_shape(int m_total, int T, int K, int batches, bool split_k) {
   GemmShape g;
   g.m_total = m_total;
   g.m_tiles = (m_total + G::BM - 1) / G::BM;
@@ -283,7 +306,7 @@ GemmShape gemm_shape(int m_total, int T, int K, int batches) {
   g.n_tiles = (T + g.n_tile - 1) / g.n_tile;
   g.k_blocks = K / G::BK;
   g.batches = batches;
-  g.splits = G::choose_splits(g.m_tiles * g.n_tiles * batches, g.k_blocks, sm_count());
+  g.splits = split_k ? G::choose_splits(g.m_tiles * g.n_tiles * batches, g.k_blocks, sm_count()) : 1;
   return g;
 }
 
@@ -291,10 +314,11 @@ size_t gemm_part_bytes(const GemmShape &g, int T) {
   return sizeof(float) * static_cast<size_t>(g.batches) * g.splits * T * g.m_total;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const GemmShape &g,
-                       int T, int m_split, bool a_mn_major, int a_batch_rows, int b_batch_cols, float *out,
+                       int T, int m_split, bool a_mn_major, int a_batch_rows, int b_batch_cols, G::Params p,
                        cudaStream_t st) {
-  G::Params p{};
   p.m_total = g.m_total;
   p.m_split = m_split;
   p.n_total = T;
@@ -306,20 +330,19 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
   p.a_batch_rows = a_batch_rows;
   p.b_batch_cols = b_batch_cols;
   p.stages = G::stages_for(g.n_tile);
-  p.out = out;
   const size_t smem = G::smem_for(g.n_tile, p.stages);
-  static size_t attr = 0;
-  if (smem > attr) {
+  static bool attr = false;
+  if (!attr) {
     if (cudaFuncSetAttribute(G::k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
       return cuda_check("gemm: set shared memory size");
-    attr = 232448;
+    attr = true;
   }
   dim3 grid(g.m_tiles, g.n_tiles, g.batches * g.splits);
   MLA_LAUNCH(G::k_gemm<<<grid, G::NUM_THREADS, smem, st>>>(ta, ta2, tb, p));
   return cuda_check("projection GEMM (tensor cores)");
 }
 
-GemmShape append_shape(const mla_dims *d, int T) { return gemm_shape(d->d_c + d->d_r, T, d->d, 1); }
+GemmShape append_shape(const mla_dims *d, int T) { return gemm_shape(d->d_c + d->d_r, T, d->d, 1, true); }
 
 size_t tc_append_ws(const mla_dims *d, int T) { return gemm_part_bytes(append_shape(d, T), T); }
 
@@ -332,28 +355,29 @@ mla_status tc_append(const mla_dims *d, const void *h, const void *W_DKV, const 
   if ((s = make_tmap_bf16(&ta2, W_KR, d->d, d->d_r, d->d * 2ull, 64, 128, "W_KR")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, g.n_tile, "h")) != MLA_OK) return s;
   float *part = static_cast<float *>(ws);
-  if ((s = launch_gemm(ta, ta2, tb, g, T, d->d_c, false, 0, 0, part, st)) != MLA_OK) return s;
-  MLA_LAUNCH(G::k_fin_append<<<T, 288, 0, st>>>(part, g.splits, T, d->d_c, d->d_r, d->rope_base, seq_idx, positions,
-                                               view_of(c)));
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = part;
+  if ((s = launch_gemm(ta, ta2, tb, g, T, d->d_c, false, 0, 0, p, st)) != MLA_OK) return s;
+  const int D = d->d_c + d->d_r;
+  MLA_LAUNCH(G::k_fin_append<<<dim3((D / 2 + 127) / 128, T), 128, 0, st>>>(part, g.splits, T, d->d_c, d->d_r,
+                                                                         d->rope_base, seq_idx, positions,
+                                                                         view_of(c)));
   return cuda_check("append finalize");
 }
 
 struct AbsorbPlan {
   GemmShape cq, uq, uk;
-  size_t part, cq_off, qc_off, total;
+  size_t cq_off, qc_off, total;
 };
 
 AbsorbPlan absorb_plan(const mla_dims *d, int T) {
   AbsorbPlan a;
-  a.cq = gemm_shape(d->d_cq, T, d->d, 1);
-  a.uq = gemm_shape(d->n_h * (d->d_h + d->d_r), T, d->d_cq, 1);
-  a.uk = gemm_shape(d->d_c, T, d->d_h, d->n_h);
-  size_t part = gemm_part_bytes(a.cq, T);
-  part = std::max(part, gemm_part_bytes(a.uq, T));
-  part = std::max(part, gemm_part_bytes(a.uk, T));
-  a.part = (part + 255) & ~size_t(255);
-  a.cq_off = a.part;
-  a.qc_off = a.cq_off + ((static_cast<size_t>(T) * d->d_cq * 2 + 255) & ~size_t(255));
+  a.cq = gemm_shape(d->d_cq, T, d->d, 1, true);
+  a.uq = gemm_shape(d->n_h * (d->d_h + d->d_r), T, d->d_cq, 1, false);
+  a.uk = gemm_shape(d->d_c, T, d->d_h, d->n_h, false);
+  a.cq_off = align256(gemm_part_bytes(a.cq, T));
+  a.qc_off = a.cq_off + align256(static_cast<size_t>(T) * d->d_cq * 2);
   a.total = a.qc_off + static_cast<size_t>(T) * d->n_h * d->d_h * 2;
   return a;
 }
@@ -367,37 +391,51 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   __nv_bfloat16 *cq = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.cq_off);
   __nv_bfloat16 *qc = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.qc_off);
   const int HD = d->n_h * d->d_h;
+  const int64_t Dq = d->d_c + d->d_r;
   CUtensorMap ta, ta2, tb;
   mla_status s;
-  // c_Q = W_DQ h
+  // c_Q = W_DQ h (split K, fp32 partials, then rounded to bf16 for the next product)
   if ((s = make_tmap_bf16(&ta, W_DQ, d->d, d->d_cq, d->d * 2ull, 64, 128, "W_DQ")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, a.cq.n_tile, "h")) != MLA_OK) return s;
-  if ((s = launch_gemm(ta, ta, tb, a.cq, T, d->d_cq, false, 0, 0, part, st)) != MLA_OK) return s;
-  MLA_LAUNCH(G::k_fin_store<<<std::max(1, std::min(1024, T * d->d_cq / 512)), 256, 0, st>>>(part, a.cq.splits, T,
-                                                                                         d->d_cq, cq, d->d_cq));
-  // [q_C ; q_R] = [W_UQ ; W_QR] c_Q, RoPE on q_R
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = part;
+  if ((s = launch_gemm(ta, ta, tb, a.cq, T, d->d_cq, false, 0, 0, p, st)) != MLA_OK) return s;
+  const int64_t pairs = static_cast<int64_t>(T) * d->d_cq / 2;
+  MLA_LAUNCH(G::k_fin_store<<<static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256)), 256, 0, st>>>(
+      part, a.cq.splits, T, d->d_cq, cq, d->d_cq));
+  // [q_C ; q_R] = [W_UQ ; W_QR] c_Q: q_C to the workspace, q_R rotated into q
   if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&ta2, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK)
     return s;
   if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, a.uq.n_tile, "c_Q")) != MLA_OK) return s;
-  if ((s = launch_gemm(ta, ta2, tb, a.uq, T, HD, false, 0, 0, part, st)) != MLA_OK) return s;
-  MLA_LAUNCH(G::k_fin_uq<<<dim3(24, T), 512, 0, st>>>(part, a.uq.splits, T, d->n_h, d->d_h, d->d_c, d->d_r,
-                                                     d->rope_base, positions, qc, static_cast<__nv_bfloat16 *>(q)));
+  p = G::Params{};
+  p.epi = G::EPI_UQ;
+  p.dst = qc;
+  p.e_split = HD;
+  p.q = static_cast<__nv_bfloat16 *>(q);
+  p.n_h = d->n_h;
+  p.d_c = d->d_c;
+  p.d_r = d->d_r;
+  p.rope_base = d->rope_base;
+  p.positions = positions;
+  if ((s = launch_gemm(ta, ta2, tb, a.uq, T, HD, false, 0, 0, p, st)) != MLA_OK) return s;
   // q_lat,h = W_UK_h^T q_C,h: A(m = latent j, k = i) = W_UK[h*d_h + i][j], m contiguous
   if ((s = make_tmap_bf16(&ta, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UK")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&tb, qc, HD, T, HD * 2ull, 64, a.uk.n_tile, "q_C")) != MLA_OK) return s;
-  if ((s = launch_gemm(ta, ta, tb, a.uk, T, d->d_c, true, d->d_h, d->d_h, part, st)) != MLA_OK) return s;
-  const int64_t D = d->d_c + d->d_r;
-  MLA_LAUNCH(G::k_fin_heads<<<dim3(std::max(1, std::min(64, T * d->d_c / 512)), d->n_h), 256, 0, st>>>(
-      part, a.uk.splits, T, d->d_c, d->n_h, static_cast<__nv_bfloat16 *>(q), d->n_h * D, D));
-  return cuda_check("absorb finalize");
+  p = G::Params{};
+  p.epi = G::EPI_BF16;
+  p.dst = static_cast<__nv_bfloat16 *>(q);
+  p.e_bs = Dq;
+  p.e_ns = d->n_h * Dq;
+  return launch_gemm(ta, ta, tb, a.uk, T, d->d_c, true, d->d_h, d->d_h, p, st);
 }
 
-GemmShape out_proj_shape(const mla_dims *d, int T) { return gemm_shape(d->d_h, T, d->d_c, d->n_h); }
+GemmShape out_proj_shape(const mla_dims *d, int T) { return gemm_shape(d->d_h, T, d->d_c, d->n_h, false); }
 
-size_t tc_out_proj_ws(const mla_dims *d, int T) { return gemm_part_bytes(out_proj_shape(d, T), T); }
+size_t tc_out_proj_ws(const mla_dims *, int) { return 0; }
 
-mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int T, void *o, void *ws,
+mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int T, void *o, void *,
                        cudaStream_t st) {
   const GemmShape g = out_proj_shape(d, T);
   const int HD = d->n_h * d->d_h, HC = d->n_h * d->d_c;
@@ -405,11 +443,12 @@ mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, i
   mla_status s;
   if ((s = make_tmap_bf16(&ta, W_UV, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UV")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&tb, o_lat, HC, T, HC * 2ull, 64, g.n_tile, "o_lat")) != MLA_OK) return s;
-  float *part = static_cast<float *>(ws);
-  if ((s = launch_gemm(ta, ta, tb, g, T, d->d_h, false, d->d_h, d->d_c, part, st)) != MLA_OK) return s;
-  MLA_LAUNCH(G::k_fin_heads<<<dim3(std::max(1, std::min(64, T * d->d_h / 512)), d->n_h), 256, 0, st>>>(
-      part, g.splits, T, d->d_h, d->n_h, static_cast<__nv_bfloat16 *>(o), HD, d->d_h));
-  return cuda_check("out_proj finalize");
+  G::Params p{};
+  p.epi = G::EPI_BF16;
+  p.dst = static_cast<__nv_bfloat16 *>(o);
+  p.e_bs = d->d_h;
+  p.e_ns = HD;
+  return launch_gemm(ta, ta, tb, g, T, d->d_h, false, d->d_h, d->d_c, p, st);
 }
 
 // ------------------------------------------------- tensor-core decode ----
@@ -447,22 +486,43 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   namespace D = mla::dec;
   const int BJ = B * n_q;
   if (BJ > D::MAX_UNITS) return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode supports B*n_q <= %d", D::MAX_UNITS);
-  if (c->paged && c->block_size % D::TILE != 0)
-    return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode needs block_size to be a multiple of %d", D::TILE);
+  if (c->paged && c->block_size % D::BLK != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode needs block_size to be a multiple of %d", D::BLK);
   const int64_t rows = c->paged ? c->num_blocks * c->block_size : static_cast<int64_t>(c->num_seqs) * c->max_len;
   if (rows >= 0x7fff0000LL) return fail(MLA_ERR_UNSUPPORTED, "cache has too many rows for 32-bit TMA coordinates");
   const int sms = sm_count();
   const int nclusters = decode_clusters(sms);
   if (ws_bytes < mla::decode_tc_ws(B, n_q, sms)) return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
 
-  CUtensorMap tm_q, tm_ks, tm_v;
+  // Views with a 128-byte column-chunk dimension (stride 128 B) inside each
+  // 1152-byte row, so one box moves a block's slab chunk-major:
+  //   q:     (64 cols, row, 9 chunks)                 box (64, 64 heads, 9)
+  //   score: (64 cols, row, 9 chunks)                 boxes (64, 64 tokens, 2) and (64, 64, 1)
+  //   value: (64 cols, row, 2 chunks, 2 halves) at column 128 * rank, half stride 256 cols
+  //          box (64, 64 tokens, 2, 1) = 128 of this CTA's latent columns
+  CUtensorMap tm_q, tm_k2, tm_k1, tm_v[2];
   mla_status s;
-  if ((s = make_tmap_bf16(&tm_q, q, D::D, static_cast<uint64_t>(BJ) * D::HEADS, D::D * 2, 64, D::HPC, "q")) != MLA_OK)
-    return s;
-  if ((s = make_tmap_bf16(&tm_ks, c->data, D::D, rows, D::D * 2, 64, D::OWN, "cache (score tile)")) != MLA_OK) return s;
-  if ((s = make_tmap_bf16(&tm_v, c->data, D::D, rows, D::D * 2, 64, D::TILE, "cache (value tile)")) != MLA_OK) return s;
+  const uint64_t row_b = D::D * 2;
+  {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(BJ) * D::HEADS, 9}, str[2] = {row_b, 128};
+    const uint32_t box[3] = {64, D::HPC, 9};
+    if ((s = make_tmap_nd(&tm_q, q, 3, dims, str, box, "q")) != MLA_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), 9}, str[2] = {row_b, 128};
+    const uint32_t box2[3] = {64, D::BLK, 2}, box1[3] = {64, D::BLK, 1};
+    if ((s = make_tmap_nd(&tm_k2, c->data, 3, dims, str, box2, "cache (score slabs)")) != MLA_OK) return s;
+    if ((s = make_tmap_nd(&tm_k1, c->data, 3, dims, str, box1, "cache (score slabs)")) != MLA_OK) return s;
+  }
+  for (int r = 0; r < 2; ++r) {
+    const uint64_t dims[4] = {64, static_cast<uint64_t>(rows), 2, 2}, str[3] = {row_b, 128, 512};
+    const uint32_t box[4] = {64, D::BLK, 2, 1};
+    const void *base = static_cast<const uint8_t *>(c->data) + 256 * r;
+    if ((s = make_tmap_nd(&tm_v[r], base, 4, dims, str, box, "cache (value slabs)")) != MLA_OK) return s;
+  }
 
   D::Params p{};
+  p.cache = static_cast<const uint8_t *>(c->data);
   p.seq_lens = seq_lens;
   p.block_table = c->block_table;
   p.max_len = c->max_len;
@@ -490,7 +550,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
       return cuda_check("decode: set shared memory size");
     attr_done = true;
   }
-  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_ks, tm_v, p));
+  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k2, tm_k1, tm_v[0], tm_v[1], p));
   if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
   MLA_LAUNCH(D::k_combine<<<BJ * 16, 256, 0, st>>>(p));
   return cuda_check("decode combine");

@@ -63,14 +63,22 @@ def test_decode_uses_tensor_cores_for_deepseek_dims(mla):
     assert not mla.uses_tensor_cores(dims_of(synth.WORKLOADS["tiny_fp32"], mla), mla.OP_DECODE)
 
 
-@pytest.mark.parametrize("seq_lens", [[1], [64], [65], [1, 2, 63, 64, 65, 127, 128, 129, 200, 1000]])
+@pytest.mark.parametrize("seq_lens", [[1], [64], [65], [256], [257],
+                                      [1, 2, 63, 64, 65, 127, 128, 129, 200, 1000],
+                                      [191, 192, 193, 255, 256, 257, 300, 511, 512, 513, 700, 769]])
 def test_decode_tc_paged_ragged(mla, orc, seq_lens):
     _run(mla, orc, V2, 11, seq_lens)
+
+
+def test_decode_tc_paged_block_128(mla, orc):
+    # blocks of 128 tokens: two 64-token value chunks per block
+    _run(mla, orc, synth.shrink(V2, block_size=128), 22, [1, 129, 300, 1000])
 
 
 def test_decode_tc_contiguous(mla, orc):
     w = synth.shrink(synth.WORKLOADS["v2_b16_4k"])
     _run(mla, orc, w, 12, [700, 33, 1500, 64])
+    _run(mla, orc, w, 21, [257, 1, 511, 130])
 
 
 def test_decode_tc_splits_long_sequences(mla, orc):
