@@ -18,6 +18,7 @@ import math
 import os
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -54,15 +55,25 @@ def parse():
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons, each stamped with the
+    host time it arrived, so that the summary keeps only the samples taken while
+    the timed region ran (mark() brackets it). The GPU is addressed by UUID,
+    which stays right under CUDA_VISIBLE_DEVICES."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id):
+        self.gpu = gpu_id
         self.proc = None
+        self.samples = []  # (host time, line)
+        self.window = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.samples.append((time.perf_counter(), line))
 
     def __enter__(self):
         try:
@@ -71,23 +82,36 @@ class ClockSampler:
                  "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        t0 = time.perf_counter()
+        while not self.samples and time.perf_counter() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)  # sampling is running before the caller starts its timed region
         return self
 
+    def mark(self, t_begin, t_end):
+        self.window = (t_begin, t_end)
+
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.reader.join(timeout=5)
 
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        lines = self.samples
+        if self.window is not None:
+            a, b = self.window
+            inside = [x for x in lines if a <= x[0] <= b]
+            # a short timed region may fall between two 20 ms samples: keep the nearest one
+            lines = inside or sorted(lines, key=lambda x: abs(x[0] - 0.5 * (a + b)))[:1]
+        for _, l in lines:
             parts = [x.strip() for x in l.split(",")]
             if len(parts) < 9:
                 continue
@@ -103,6 +127,15 @@ class ClockSampler:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def gpu_id_for_smi(torch, local_rank):
+    """nvidia-smi id of this process's CUDA device (its UUID when torch exposes it)."""
+    try:
+        u = str(torch.cuda.get_device_properties(local_rank).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local_rank)
 
 
 # ----------------------------------------------------------------- our arm --
@@ -173,12 +206,14 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     launches0 = mla.kernel_launches()
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(gpu_id_for_smi(torch, local_rank)) as clk:
+        h0 = time.perf_counter()
         t0.record(stream)
         for i in range(args.steps):
             step(i)
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark(h0, time.perf_counter())
     launches = mla.kernel_launches() - launches0
     barrier()
     ms_total = t0.elapsed_time(t1)

@@ -12,30 +12,31 @@
 //    pair of SMs (a 2-CTA cluster) with M = 128, N = 256: CTA r holds heads
 //    64r..64r+63 of Q, supplies tokens 128r..128r+127 of the tile to QK^T
 //    (B split by N = tokens) and latent columns [256j + 128r, +128) of every
-//    token to PV (B split by N = latent). Each MMA instruction then carries
-//    512K flop per SM, enough to keep the tensor pipe fed from one issuing
-//    thread (a tcgen05.mma takes ~25 ns to issue whatever its size).
+//    token to PV (B split by N = latent). The tensor pipe retires one MMA
+//    instruction per ~35 ns whatever its shape, and only M128 x N256 pair
+//    instructions carry a full 35 ns of work, so both products use that shape
+//    (68 instructions per tile).
 //  * The 128 x 512 fp32 accumulator O is one whole SM of tensor memory, so it
 //    is split over the pair: 256 columns per CTA, plus two 128-column score
 //    buffers = all 512 columns.
-//  * Shared memory per CTA: Q 72 KB resident per piece, P 32 KB, and one
-//    7-slot ring of 16 KB slabs consumed strictly in MMA order: the score
-//    slabs of tile i + 1 (per own block: 4 slabs of 2 column chunks + 1 of
-//    the last chunk), then the value slabs of tile i (per block: 2 slabs of
-//    128 latent columns). One ring for both operands keeps every slot in
-//    flight whichever product the tensor pipe is on. Latent columns are read
-//    twice from L2 (once per operand); HBM sees each cached row once.
-//  * Loads: 3-D / 4-D tensor maps view the cache as (64 columns, row, column
-//    chunk [, latent half]) with the chunk stride (128 B) smaller than the row
-//    stride, so one TMA instruction moves a whole 24-72 KB slab of a block
-//    straight into the chunk-major 128-byte-swizzled layout the MMAs read.
-//    (Many small 64 x 64 boxes cap TMA well below HBM bandwidth.)
-//  * QK^T is issued as N = 128 MMAs (64 tokens = one block per CTA) so each
-//    B operand is one contiguous block slab; PV uses N = 256 (latent).
-//  * Warp roles: warp 0 loads Q and fills the ring, warp 1 of CTA 0 issues
-//    the MMAs of the pair, warps 2-5 of both CTAs run the online softmax
-//    (fp32, exp2, O rescaled only when the running max grows by more than
-//    2^8) and the epilogue.
+//  * Shared memory per CTA: Q 72 KB resident per piece, P 32 KB, and a ring
+//    of three 32 KB slots and one 16 KB slot consumed strictly in MMA order:
+//    the score operands of tile i + 1 (column chunks {0,1} {2,3} {4,5} {6,7}
+//    in big slots, chunk 8 in the small one; each chunk holds this CTA's 128
+//    tokens as 128 rows so that one N = 256 MMA spans them), then the value
+//    operands of tile i (one big slot per 64-token block: 256 of this CTA's
+//    latent columns). Every ring item costs a commit (~70 ns of tensor-pipe
+//    time), so items are as large as the shared memory allows. Latent columns
+//    are read twice from L2 (once per operand); HBM sees each cached row
+//    once, brought into L2 by a whole-block prefetch two tiles ahead.
+//  * Loads: a TMA instruction occupies its issuing warp for ~0.3 us whatever
+//    the box size (the lanes of a warp issue in parallel), so three producer
+//    warps share the ring, big slot s belonging to warp s and the small slot
+//    and Q to warp 0: every slot's uses are issued in order by one warp, whose
+//    lanes issue an item's boxes together.
+//  * Warp roles: warps 0-2 load, warp 3 of CTA 0 issues the MMAs of the pair,
+//    warps 4-7 of both CTAs run the online softmax (fp32, exp2, O rescaled
+//    only when the running max grows by more than 2^8) and the epilogue.
 //  * Work: the visible 256-token tiles of all token rows are concatenated and
 //    cut into equal contiguous ranges, one per cluster (persistent grid). A
 //    row whose tiles fall in one range is finished in place (bf16 o_lat,
@@ -53,39 +54,53 @@ namespace mla {
 namespace dec {
 
 constexpr int D = 576, DC = 512, DR = 64, HEADS = 128, HPC = 64;
-constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CTA / per value chunk
-constexpr int NR = 7;                           // ring slots
-constexpr int NUM_THREADS = 192;                // 6 warps, see the role list in k_decode
+constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CTA / per block
+// 8 warps = 2 per SM sub-partition, so each thread may hold up to 255 registers
+constexpr int NUM_PRODUCERS = 3, WARP_MMA = 3, WARP_SOFTMAX = 4;
+constexpr int NUM_THREADS = 32 * (WARP_SOFTMAX + 4);
+constexpr int NBIG = NUM_PRODUCERS;  // 32 KB ring slots; big slot s belongs to producer warp s
+constexpr int SMALL_OWNER = 0, Q_OWNER = 0;
 constexpr int CHUNK_Q = HPC * 128;   // 64 heads x 64 columns
-constexpr int ATOM_V = BLK * 128;    // 64 tokens x 64 columns (one 128-byte-swizzle atom column)
-constexpr int SLOT = 2 * ATOM_V;     // ring slot: 2 atoms
-constexpr int K_SLABS = 5;           // per own block: chunks {0,1} {2,3} {4,5} {6,7} {8}
-constexpr int LOADS_PER_TILE = 2 * K_SLABS + 4 * 2;  // score slabs (2 own blocks) + value slabs
+constexpr int ATOM = BLK * 128;      // 64 rows x 64 columns (one 128-byte-swizzle atom column)
+constexpr int CHUNK_K = 2 * ATOM;    // one column chunk of the CTA's 128 tokens
+constexpr int BIG = 4 * ATOM, SMALL = 2 * ATOM, HALF = BIG / 2;
+constexpr int K_ITEMS = 5, V_ITEMS = 4;  // per tile: chunks {0,1} {2,3} {4,5} {6,7} {8}; one per block
+constexpr int BIG_PER_TILE = 8;          // big-slot uses per tile (4 score + 4 value items)
 constexpr int CHUNK_P = HPC * 128;   // 64 heads x 64 tokens
 constexpr int Q_BYTES = 9 * CHUNK_Q;
 constexpr int P_BYTES = 4 * CHUNK_P;
 constexpr int OFF_Q = 0;
 constexpr int OFF_P = OFF_Q + Q_BYTES;
-constexpr int OFF_R = OFF_P + P_BYTES;
-constexpr int OFF_MISC = OFF_R + NR * SLOT;
-constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_R_FULL = 2, BAR_R_EMPTY = BAR_R_FULL + NR,
-              BAR_V_LANDED = BAR_R_EMPTY + NR, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
-              BAR_S_FREE = BAR_S_FULL + 2,
-              BAR_P_FULL = BAR_S_FREE + 2, BAR_O_FULL = BAR_P_FULL + 1, BAR_O_FREE = BAR_O_FULL + 1,
-              BAR_EXIT = BAR_O_FREE + 1, NUM_BARS = BAR_EXIT + 1;
+constexpr int OFF_BIG = OFF_P + P_BYTES;
+constexpr int OFF_SMALL = OFF_BIG + NBIG * BIG;
+constexpr int OFF_MISC = OFF_SMALL + SMALL;
+constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_BIG_FULL = 2, BAR_BIG_EMPTY = BAR_BIG_FULL + NBIG,
+              BAR_SMALL_FULL = BAR_BIG_EMPTY + NBIG, BAR_SMALL_EMPTY = BAR_SMALL_FULL + 1,
+              BAR_V_LANDED = BAR_SMALL_EMPTY + 1, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
+              BAR_S_FREE = BAR_S_FULL + 2, BAR_P_FULL = BAR_S_FREE + 2, BAR_O_FULL = BAR_P_FULL + 1,
+              BAR_O_FREE = BAR_O_FULL + 1, BAR_EXIT = BAR_O_FREE + 1, NUM_BARS = BAR_EXIT + 1;
 constexpr int MISC_RED = 256;               // float red[2][128]
 constexpr int MISC_REDL = MISC_RED + 1024;  // float redl[128]
-constexpr int PF_TILES = 2;                 // L2 prefetch distance in tiles
 constexpr int MISC_INTS = MISC_REDL + 512;
 constexpr int MISC_BYTES = MISC_INTS + 64;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr int PF_TILES = 2;                                // L2 prefetch distance in tiles
 static_assert(NUM_BARS * 8 <= MISC_RED, "barriers overlap the exchange arrays");
 static_assert(SMEM_BYTES <= 232448, "decode shared memory budget");
-constexpr int MAX_UNITS = NR * SLOT / 4 - 1;  // plan scratch aliases the ring
-constexpr int S_COL = 256;                        // TMEM: O at [0,256), scores at [256 + 128 b, +128)
-constexpr uint32_t IDESC_S = idesc_bf16(128, 2 * BLK, false, false);  // N = one block per CTA
+static_assert(OFF_P % 1024 == 0 && OFF_BIG % 1024 == 0 && OFF_SMALL % 1024 == 0, "128-byte swizzle alignment");
+constexpr int MAX_UNITS = (NBIG * BIG + SMALL) / 4 - 1;  // plan scratch aliases the ring
+constexpr int S_COL = 256;                    // TMEM: O at [0,256), scores at [256 + 128 b, +128)
+constexpr uint32_t IDESC_S = idesc_bf16(128, 256, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
 constexpr float RESCALE_LOG2 = 8.f;
+
+// Ring items in MMA consumption order, per piece of n tiles: the score items
+// of tile 0; for every later tile its score items followed by the value items
+// of the tile before it; the value items of the last tile. The big-slot use
+// of the value item (tile i, block v) of a piece:
+__host__ __device__ constexpr int value_item(int i, int n, int v) {
+  return 4 * (i + 2 < n ? i + 2 : n) + 4 * i + v;
+}
 
 struct Params {
   const uint8_t *cache;  // base of the cache rows (L2 prefetch addresses)
@@ -183,8 +198,8 @@ __device__ __forceinline__ void arrive_leader(uint32_t bar_local, uint32_t rank)
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
-    k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k2,
-             const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_v0,
+    k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_pf, const __grid_constant__ CUtensorMap tm_v0,
              const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -206,10 +221,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
     mbar_init(bar(BAR_Q_EMPTY), 1);
-    for (int s = 0; s < NR; ++s) {
-      mbar_init(bar(BAR_R_FULL + s), 1);
-      mbar_init(bar(BAR_R_EMPTY + s), 1);
+    for (int s = 0; s < NBIG; ++s) {
+      mbar_init(bar(BAR_BIG_FULL + s), 1);
+      mbar_init(bar(BAR_BIG_EMPTY + s), 1);
     }
+    mbar_init(bar(BAR_SMALL_FULL), 1);
+    mbar_init(bar(BAR_SMALL_EMPTY), 1);
     mbar_init(bar(BAR_V_LANDED), 1);
     mbar_init(bar(BAR_ZERO_DONE), 8);
     for (int b = 0; b < 2; ++b) {
@@ -224,17 +241,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     fence_mbar_init();
   }
   const CUtensorMap *tm_v = rank == 0 ? &tm_v0 : &tm_v1;  // value slabs: this CTA's latent columns
-  if (warp == 0) {
+  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k2);
-    tma_prefetch_desc(&tm_k1);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_pf);
     tma_prefetch_desc(tm_v);
   }
-  if (warp == 1) tmem_alloc<2>(smem_u32(tmem_slot), 512);
+  if (warp == WARP_MMA) tmem_alloc<2>(smem_u32(tmem_slot), 512);
 
   // ---- plan: tiles per unit, prefix sums, this cluster's first unit ----
   const int BJ = p.B * p.n_q;
-  int *scratch = reinterpret_cast<int *>(smem + OFF_R);
+  int *scratch = reinterpret_cast<int *>(smem + OFF_BIG);
   for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
     int vis;
     int nt = unit_tiles(p, u, &vis);
@@ -309,120 +326,172 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   it0.Qt = Qt;
   it0.k = cluster;
 
-  if (warp == 0) {
-    // --------------------------------------------------------- ring producer
-    // Load order = MMA consumption order: per piece Q, then score slabs of
-    // tile 0, and for every later tile its score slabs followed by the value
-    // slabs of the tile before it; the last tile's value slabs close the
-    // piece. Block rows of a tile are read one tile before they are needed.
-    if (lane == 0) {
-      const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
-      PieceIter it = it0;
-      Piece pc;
-      int g = 0, npc = 0;
-      bool ok = true;
-      auto slot_for_load = [&](uint32_t bytes) -> int {  // wait for a free slot, arm its barrier
-        const int s = g % NR;
-        if (g >= NR && !mbar_wait(bar(BAR_R_EMPTY + s), ((g / NR) - 1) & 1, abort_flag)) return -1;
-        if (rank == 0) mbar_arrive_expect_tx(bar(BAR_R_FULL + s), 2 * bytes);
-        return s;
+  if (warp < NUM_PRODUCERS) {
+    // --------------------------------------------------------- ring producers
+    // Every producer warp walks the same item sequence and issues the items
+    // of the slots it owns, so that each slot's uses are issued in order by
+    // one warp (a parity wait on the slot's empty barrier is exact only when
+    // the waiter is at most one phase ahead). Lane 0 waits for the slot and
+    // arms its full barrier, then lane l issues box l of the item. The L2
+    // prefetch of tile t goes to warp t mod NUM_PRODUCERS.
+    const int w = warp;
+    const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
+    PieceIter it = it0;
+    Piece pc;
+    int nbig = 0, nsmall = 0, npc = 0, ntile = 0;
+    bool ok = true;
+    auto full_of = [&](int bi) { return rank == 0 ? bar(bi) : mapa_shared(bar(bi), 0); };
+    // Next item: 0 if another warp issues it; else waits for its slot, arms
+    // the barrier (*fb) and returns the slot's shared-memory offset, or -1 on
+    // a failed wait (all warp-uniform).
+    auto claim = [&](bool big, uint32_t bytes, int *fb) -> int {
+      int slot, use;
+      if (big) {
+        slot = nbig % NBIG;
+        use = nbig / NBIG;
+        ++nbig;
+      } else {
+        slot = 0;
+        use = nsmall++;
+      }
+      if ((big ? slot : SMALL_OWNER) != w) return 0;
+      const int eb = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
+      *fb = big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL;
+      bool good = true;
+      if (lane == 0) {
+        if (use > 0) good = mbar_wait(bar(eb), (use - 1) & 1, abort_flag);
+        if (good && rank == 0) mbar_arrive_expect_tx(bar(*fb), 2 * bytes);
+      }
+      return __shfl_sync(0xffffffffu, good, 0) ? (big ? OFF_BIG + slot * BIG : OFF_SMALL) : -1;
+    };
+    auto load_k = [&](const int32_t *own) -> bool {  // score items of one tile (own blocks)
+      for (int q = 0; q < K_ITEMS; ++q) {
+        const bool big = q < K_ITEMS - 1;
+        int fb = 0;
+        const int off = claim(big, big ? BIG : SMALL, &fb);
+        if (off < 0) return false;
+        if (off == 0) continue;
+        if (lane < (big ? 4 : 2)) {  // lane l: column chunk 2q + l / 2 of own block l % 2
+          const int c = 2 * q + (lane >> 1), kb = lane & 1;
+          tma_load_2d_pair(sbase + off + (lane >> 1) * CHUNK_K + kb * ATOM, &tm_k, 64 * c, own[kb], full_of(fb));
+        }
+        __syncwarp();
+      }
+      return true;
+    };
+    auto load_v = [&](const int32_t *rows) -> bool {  // value items of one tile: block v, both latent halves
+      for (int v = 0; v < 4; ++v) {
+        int fb = 0;
+        const int off = claim(true, BIG, &fb);
+        if (off < 0) return false;
+        if (off == 0) continue;
+        if (lane < 2)  // lane j: latent half j (16 KB)
+          tma_load_4d_pair(sbase + off + lane * HALF, tm_v, 0, rows[v], 0, lane, full_of(fb));
+        __syncwarp();
+      }
+      return true;
+    };
+    while (ok && it.next(p, pc)) {
+      const int b = pc.bj / p.n_q;
+      auto rows_of = [&](int ti, int32_t *r4) {
+        for (int v = 0; v < 4; ++v) r4[v] = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * v, pc.vis);
       };
-      auto full_of = [&](int s) { return rank == 0 ? bar(BAR_R_FULL + s) : mapa_shared(bar(BAR_R_FULL + s), 0); };
-      auto load_k = [&](const int32_t *own) -> bool {  // score slabs of one tile (own blocks)
-        for (int kb = 0; kb < 2; ++kb)
-          for (int m = 0; m < K_SLABS; ++m) {
-            const bool last = m == K_SLABS - 1;
-            const int s = slot_for_load(last ? ATOM_V : SLOT);
-            if (s < 0) return false;
-            tma_load_3d_pair(sbase + OFF_R + s * SLOT, last ? &tm_k1 : &tm_k2, 0, own[kb], 2 * m, full_of(s));
-            ++g;
+      auto prefetch = [&](int ti) {  // whole own blocks of tile ti into L2 (lanes 0, 1)
+        if (lane < 2) {
+          const int32_t r = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * (2 * rank + lane), pc.vis);
+          if (r < p.cache_rows) tma_prefetch_3d(&tm_pf, 0, r, 0);
+        }
+        __syncwarp();
+      };
+      int32_t cur[4], prev[4], nxt[4];
+      rows_of(pc.t_begin, cur);
+      for (int ti = pc.t_begin; ti < min(pc.t_end, pc.t_begin + PF_TILES); ++ti)
+        if (((ntile + ti - pc.t_begin) % NUM_PRODUCERS) == w) prefetch(ti);
+      if (w == Q_OWNER) {
+        bool good = true;
+        if (lane == 0) {
+          if (npc > 0) good = mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
+          if (good) {
+            if (rank == 0) mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * Q_BYTES);
+            tma_load_3d_pair(sbase + OFF_Q, &tm_q, 0, pc.bj * HEADS + HPC * rank, 0, q_full);
           }
-        return true;
-      };
-      auto load_v = [&](const int32_t *rows) -> bool {  // value slabs of one tile (all 4 blocks)
-        for (int v = 0; v < 4; ++v)
-          for (int j = 0; j < 2; ++j) {
-            const int s = slot_for_load(SLOT);
-            if (s < 0) return false;
-            tma_load_4d_pair(sbase + OFF_R + s * SLOT, tm_v, 0, rows[v], 0, j, full_of(s));
-            ++g;
-          }
-        return true;
-      };
-      while (ok && it.next(p, pc)) {
-        const int b = pc.bj / p.n_q;
-        auto rows_of = [&](int ti, int32_t *r4) {
-          for (int v = 0; v < 4; ++v) r4[v] = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * v, pc.vis);
-        };
-        int32_t cur[4], prev[4], nxt[4];
-        rows_of(pc.t_begin, cur);
-        if (npc > 0 && !mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag)) {
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) {
           ok = false;
           break;
         }
-        if (rank == 0) mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * Q_BYTES);
-        tma_load_3d_pair(sbase + OFF_Q, &tm_q, 0, pc.bj * HEADS + HPC * rank, 0, q_full);
-        for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti) {
-          if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
-          const int32_t own[2] = {cur[2 * rank], cur[2 * rank + 1]};
-          if (!load_k(own)) { ok = false; break; }
-          if (ti > pc.t_begin && !load_v(prev)) { ok = false; break; }
-          for (int v = 0; v < 4; ++v) {
-            prev[v] = cur[v];
-            cur[v] = nxt[v];
-          }
-        }
-        if (!ok || !load_v(prev)) { ok = false; break; }
-        ++npc;
       }
-      // drain: every commit aimed at this CTA's empty barriers has landed
-      if (ok && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
-      for (int q = g - NR; ok && q < g; ++q)
-        if (q >= 0) mbar_wait(bar(BAR_R_EMPTY + q % NR), (q / NR) & 1, abort_flag);
+      for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti, ++ntile) {
+        if (ti + PF_TILES < pc.t_end && ((ntile + PF_TILES) % NUM_PRODUCERS) == w) prefetch(ti + PF_TILES);
+        if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
+        const int32_t own[2] = {cur[2 * rank], cur[2 * rank + 1]};
+        if (!load_k(own)) { ok = false; break; }
+        if (ti > pc.t_begin && !load_v(prev)) { ok = false; break; }
+        for (int v = 0; v < 4; ++v) {
+          prev[v] = cur[v];
+          cur[v] = nxt[v];
+        }
+      }
+      if (!ok || !load_v(prev)) { ok = false; break; }
+      ++npc;
     }
-  } else if (warp == 1) {
+    // drain: every commit aimed at the empty barriers of this warp's slots
+    // (and of Q) has landed; each warp waits only on what it owns, see above
+    if (lane == 0) {
+      const int uses = nbig > w ? (nbig - w + NBIG - 1) / NBIG : 0;
+      if (ok && uses > 0) mbar_wait(bar(BAR_BIG_EMPTY + w), (uses - 1) & 1, abort_flag);
+      if (ok && w == SMALL_OWNER && nsmall > 0) mbar_wait(bar(BAR_SMALL_EMPTY), (nsmall - 1) & 1, abort_flag);
+      if (ok && w == Q_OWNER && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
+    }
+  } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0) {
       PieceIter it = it0;
       Piece pc{};
-      int gi = 0, g = 0, gz = 0, npc = 0;
+      int gi = 0, nbig = 0, nsmall = 0, gz = 0, npc = 0, empty_bar = 0;
       bool ok = true;
-      auto take = [&]() -> int {  // next ring slot in consumption order, once it has landed
-        const int s = g % NR;
-        if (!mbar_wait(bar(BAR_R_FULL + s), (g / NR) & 1, abort_flag)) return -1;
+      auto take = [&](bool big) -> uint32_t {  // next ring item in consumption order, once it has landed
+        int slot, use;
+        if (big) {
+          slot = nbig % NBIG;
+          use = nbig / NBIG;
+          ++nbig;
+        } else {
+          slot = 0;
+          use = nsmall++;
+        }
+        empty_bar = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
+        if (!mbar_wait(bar(big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL), use & 1, abort_flag)) return 0;
         tc_fence_after();
-        return s;
+        return sbase + (big ? OFF_BIG + slot * BIG : OFF_SMALL);
       };
-      auto release = [&](int s) {
-        tc_commit_pair(bar(BAR_R_EMPTY + s), 0x3);
-        ++g;
-      };
+      auto release = [&]() { tc_commit_pair(bar(empty_bar), 0x3); };
       // PV of global tile gt (tile ti of the current piece)
       auto issue_pv = [&](int gt, int ti, bool first) -> bool {
         const int zc = partial_chunk(pc.vis, ti);
-        for (int v = 0; v < 4; ++v)
-          for (int j = 0; j < 2; ++j) {
-            const int s = take();
-            if (s < 0) return false;
-            if (v == 0 && j == 0) {
-              if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
-              if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
-            }
-            if (v == zc) {  // both CTAs zero the rows past the end of this slab first
-              mbar_arrive(bar(BAR_V_LANDED));
-              mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
-              if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
-              ++gz;
-              tc_fence_after();
-            }
-            const uint32_t pa = sbase + OFF_P + v * CHUNK_P;
-            const uint32_t vb = sbase + OFF_R + s * SLOT;
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t vb = take(true);
+          if (vb == 0) return false;
+          if (v == 0) {
+            if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
+            if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+          }
+          if (v == zc) {  // both CTAs zero the rows past the end of this slab first
+            mbar_arrive(bar(BAR_V_LANDED));
+            mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
+            if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
+            ++gz;
+            tc_fence_after();
+          }
+          const uint32_t pa = sbase + OFF_P + v * CHUNK_P;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc_mma<2>(tmem + 128 * j, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(vb + kk * 2048, ATOM_V, 1024),
+              tc_mma<2>(tmem + 128 * j, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(vb + j * HALF + kk * 2048, ATOM, 1024),
                         IDESC_PV, (first && v == 0 && kk == 0) ? 0u : 1u);
-            release(s);
-          }
+          release();
+        }
         tc_commit_pair(bar(BAR_O_FULL), 0x3);
         return true;
       };
@@ -432,21 +501,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         for (int i = 0; i < n && ok; ++i, ++gi) {
           const int b = gi & 1;
           if (gi >= 2 && !mbar_wait(bar(BAR_S_FREE + b), ((gi >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-          for (int kb = 0; kb < 2 && ok; ++kb)
-            for (int m = 0; m < K_SLABS; ++m) {
-              const int s = take();
-              if (s < 0) { ok = false; break; }
-              const uint32_t slab = sbase + OFF_R + s * SLOT;
-              const int nch = m == K_SLABS - 1 ? 1 : 2;
-              for (int c = 0; c < nch; ++c)
+          for (int q = 0; q < K_ITEMS; ++q) {
+            const bool big = q < K_ITEMS - 1;
+            const uint32_t kbuf = take(big);
+            if (kbuf == 0) { ok = false; break; }
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  tc_mma<2>(tmem + S_COL + 128 * b + 64 * kb,
-                            sdesc_sw128(sbase + OFF_Q + (2 * m + c) * CHUNK_Q + kk * 32, 16, 1024),
-                            sdesc_sw128(slab + c * ATOM_V + kk * 32, 16, 1024), IDESC_S,
-                            (m > 0 || c > 0 || kk > 0) ? 1u : 0u);
-              release(s);
+            for (int c = 0; c < 2; ++c) {
+              if (!big && c == 1) break;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc_mma<2>(tmem + S_COL + 128 * b, sdesc_sw128(sbase + OFF_Q + (2 * q + c) * CHUNK_Q + kk * 32, 16, 1024),
+                          sdesc_sw128(kbuf + c * CHUNK_K + kk * 32, 16, 1024), IDESC_S, (q > 0 || c > 0 || kk > 0) ? 1u : 0u);
             }
+            release();
+          }
           if (!ok) break;
           tc_commit_pair(bar(BAR_S_FULL + b), 0x3);
           if (i == n - 1) tc_commit_pair(bar(BAR_Q_EMPTY), 0x3);
@@ -457,7 +525,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         ++npc;
       }
     }
-  } else if (warp >= 2 && warp <= 5) {
+  } else if (warp >= WARP_SOFTMAX) {
     // ------------------------------------------------- softmax + epilogue
     // A failed (timed-out) wait does not break these loops: every softmax
     // warp keeps the same sequence of named-barrier syncs and runs to the
@@ -469,7 +537,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     const float c2 = p.scale_log2;
     PieceIter it = it0;
     Piece pc;
-    int gi = 0, gz = 0, gbase = 0;  // gbase: ring loads before this piece
+    int gi = 0, gz = 0, bbase = 0;  // bbase: big-slot uses before this piece
     while (it.next(p, pc)) {
       const int n = pc.t_end - pc.t_begin;
       float m_ref = -INFINITY, lsum = 0.f;
@@ -552,29 +620,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
           *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_leader(bar(BAR_P_FULL), rank);
-        // partial block of the last tile: zero value rows past the end in its
-        // two slabs (the MMA thread signals each one as it reaches it)
+        // partial block of the last tile: zero its value rows past the end
+        // (the MMA thread signals when that slab has landed)
         const int zc = partial_chunk(pc.vis, ti);
         if (zc >= 0) {
-          // ring index of this tile's value slabs (see the producer's order)
-          const int kt = i, nt_p = n;
-          const int gv = gbase + K_SLABS * 2 * min(kt + 2, nt_p) + 8 * kt + 2 * zc;
           const int valid = vis_t - BLK * zc;
           const int nrow = BLK - valid;
-          for (int j = 0; j < 2; ++j) {
-            mbar_wait_warp(bar(BAR_V_LANDED), gz & 1, abort_flag);
-            ++gz;
-            uint8_t *vb = smem + OFF_R + ((gv + j) % NR) * SLOT;
-            for (int e = L; e < nrow * 2 * 8; e += 128) {
-              const int r = valid + e / 16, a = (e >> 3) & 1, w16 = e & 7;
-              *reinterpret_cast<uint4 *>(vb + a * ATOM_V + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) arrive_leader(bar(BAR_ZERO_DONE), rank);
+          mbar_wait_warp(bar(BAR_V_LANDED), gz & 1, abort_flag);
+          ++gz;
+          uint8_t *vb = smem + OFF_BIG + ((bbase + value_item(i, n, zc)) % NBIG) * BIG;
+          // slab = [latent half j][chunk a][64 rows][128 B]: 32 16-byte words per row
+          for (int e = L; e < nrow * 32; e += 128) {
+            const int r = valid + e / 32, j = (e >> 4) & 1, a = (e >> 3) & 1, w16 = e & 7;
+            *reinterpret_cast<uint4 *>(vb + j * HALF + a * ATOM + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) arrive_leader(bar(BAR_ZERO_DONE), rank);
         }
       }
       // ---------------------------------------------------------- epilogue
@@ -621,7 +686,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(bar(BAR_O_FREE), rank);
-      gbase += LOADS_PER_TILE * n;
+      bbase += BIG_PER_TILE * n;
     }
   }
 
@@ -634,7 +699,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   }
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc<2>(tmem, 512);
+  if (warp == WARP_MMA) tmem_dealloc<2>(tmem, 512);
 }
 
 // Merge the split partials of every token row that was cut by cluster range

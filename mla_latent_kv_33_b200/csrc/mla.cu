@@ -494,13 +494,13 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   const int nclusters = decode_clusters(sms);
   if (ws_bytes < mla::decode_tc_ws(B, n_q, sms)) return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
 
-  // Views with a 128-byte column-chunk dimension (stride 128 B) inside each
-  // 1152-byte row, so one box moves a block's slab chunk-major:
-  //   q:     (64 cols, row, 9 chunks)                 box (64, 64 heads, 9)
-  //   score: (64 cols, row, 9 chunks)                 boxes (64, 64 tokens, 2) and (64, 64, 1)
-  //   value: (64 cols, row, 2 chunks, 2 halves) at column 128 * rank, half stride 256 cols
-  //          box (64, 64 tokens, 2, 1) = 128 of this CTA's latent columns
-  CUtensorMap tm_q, tm_k2, tm_k1, tm_v[2];
+  // Views of q and the cache (rows of 576 bf16 = 1152 bytes):
+  //   q:        (64 cols, row, 9 chunks of 128 B)        box (64, 64 heads, 9)
+  //   score:    (576 cols, row)                          box (64, 64 tokens): one column chunk of a block
+  //   prefetch: (64 cols, row, 9 chunks)                 box (64, 64, 9): a whole block into L2
+  //   value:    (64 cols, row, 2 chunks, 2 halves) at column 128 * rank, half stride 256 cols
+  //             box (64, 64 tokens, 2, 1) = 128 of this CTA's latent columns of a block
+  CUtensorMap tm_q, tm_k, tm_pf, tm_v[2];
   mla_status s;
   const uint64_t row_b = D::D * 2;
   {
@@ -509,10 +509,14 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
     if ((s = make_tmap_nd(&tm_q, q, 3, dims, str, box, "q")) != MLA_OK) return s;
   }
   {
+    const uint64_t dims[2] = {static_cast<uint64_t>(D::D), static_cast<uint64_t>(rows)}, str[1] = {row_b};
+    const uint32_t box[2] = {64, D::BLK};
+    if ((s = make_tmap_nd(&tm_k, c->data, 2, dims, str, box, "cache (score chunks)")) != MLA_OK) return s;
+  }
+  {
     const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), 9}, str[2] = {row_b, 128};
-    const uint32_t box2[3] = {64, D::BLK, 2}, box1[3] = {64, D::BLK, 1};
-    if ((s = make_tmap_nd(&tm_k2, c->data, 3, dims, str, box2, "cache (score slabs)")) != MLA_OK) return s;
-    if ((s = make_tmap_nd(&tm_k1, c->data, 3, dims, str, box1, "cache (score slabs)")) != MLA_OK) return s;
+    const uint32_t box[3] = {64, D::BLK, 9};
+    if ((s = make_tmap_nd(&tm_pf, c->data, 3, dims, str, box, "cache (block prefetch)")) != MLA_OK) return s;
   }
   for (int r = 0; r < 2; ++r) {
     const uint64_t dims[4] = {64, static_cast<uint64_t>(rows), 2, 2}, str[3] = {row_b, 128, 512};
@@ -550,7 +554,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
       return cuda_check("decode: set shared memory size");
     attr_done = true;
   }
-  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k2, tm_k1, tm_v[0], tm_v[1], p));
+  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k, tm_pf, tm_v[0], tm_v[1], p));
   if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
   MLA_LAUNCH(D::k_combine<<<BJ * 16, 256, 0, st>>>(p));
   return cuda_check("decode combine");

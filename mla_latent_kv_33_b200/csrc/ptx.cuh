@@ -186,6 +186,12 @@ __device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int32_t x, int
                : "memory");
 }
 
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(x), "r"(y),
+               "r"(z)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 // Shared-memory matrix descriptor, 128-byte swizzle. Addresses/offsets in bytes.
@@ -248,6 +254,27 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // D(tmem) (+)= A(smem) * B(smem)^T ; accumulate selects D += vs D =.
+// D (tmem) [+]= A (tmem) * B (smem descriptor). For cta_group::2 with M = 128 the
+// A tile of each CTA (64 rows x 16) sits in 8 columns: row m's k = 0..7 in
+// lane m, columns 0..3, and k = 8..15 in lane m + 64, columns 4..7 (bf16 pairs).
+template <int CG>
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  if constexpr (CG == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
 template <int CG>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -286,6 +313,13 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 4 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 
 // 32 consecutive 32-bit columns of this thread's lane.
