@@ -178,10 +178,19 @@ def run_ours(args, rank, world, local_rank):
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
 
+    # the cache append and the query absorption are independent: the append
+    # runs on a side stream, joined before the decode reads the cache
+    side = torch.cuda.Stream(device=dev)
+    ev_fork, ev_join = torch.cuda.Event(), torch.cuda.Event()
+
     def step(i=None):
-        mla.mla_cache_append(p, h, W["W_DKV"], W["W_KR"], sidx, pos, cache, ws=ws[mla.OP_APPEND], stream=stream)
+        ev_fork.record(stream)
+        side.wait_event(ev_fork)
+        mla.mla_cache_append(p, h, W["W_DKV"], W["W_KR"], sidx, pos, cache, ws=ws[mla.OP_APPEND], stream=side)
+        ev_join.record(side)
         mla.mla_absorb_q(p, h, W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], pos, q, ws=ws[mla.OP_ABSORB],
                          stream=stream)
+        stream.wait_event(ev_join)
         if i is not None:
             ev_dec[i][0].record(stream)
         mla.mla_decode(p, q, cache, sl, w.n_q, o_lat, lse, ws=ws[mla.OP_DECODE], stream=stream)

@@ -44,19 +44,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// RoPE rotation of the interleaved pair (x0, x1) = (x[2i], x[2i+1]) by the
-// angle pos * base^(-2i/d_r). The angle is formed and reduced in double so
-// positions up to 2^17 and beyond keep full fp32 accuracy.
-__device__ __forceinline__ void rope_pair(float &x0, float &x1, int pair, int d_r, int pos,
-                                          double base) {
-  const double theta = pow(base, -2.0 * static_cast<double>(pair) / static_cast<double>(d_r));
-  double s, c;
-  sincos(static_cast<double>(pos) * theta, &s, &c);
-  const float cf = static_cast<float>(c), sf = static_cast<float>(s);
-  const float y0 = x0 * cf - x1 * sf;
-  const float y1 = x0 * sf + x1 * cf;
+// RoPE (RoFormer, interleaved pairs): the pair (x0, x1) = (x[2i], x[2i+1]) is
+// rotated by the angle pos * theta_i, theta_i = base^(-2i/d_r).
+__device__ __forceinline__ double rope_theta(int pair, int d_r, double base) {
+  return exp2(-2.0 * static_cast<double>(pair) / static_cast<double>(d_r) * log2(base));
+}
+
+// The angle is formed and reduced to [-pi, pi] in double (so positions up to
+// 2^17 and beyond keep full accuracy), then sine and cosine are taken in fp32.
+__device__ __forceinline__ void rope_rotate(float &x0, float &x1, int pos, double theta) {
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  const double a = static_cast<double>(pos) * theta;
+  const double k = rint(a * (1.0 / kTwoPi));
+  float s, c;
+  sincosf(static_cast<float>(fma(-k, kTwoPi, a)), &s, &c);
+  const float y0 = x0 * c - x1 * s;
+  const float y1 = x0 * s + x1 * c;
   x0 = y0;
   x1 = y1;
+}
+
+__device__ __forceinline__ void rope_pair(float &x0, float &x1, int pair, int d_r, int pos, double base) {
+  rope_rotate(x0, x1, pos, rope_theta(pair, d_r, base));
 }
 
 // Physical cache row of logical (b, pos); returns -1 when out of range.

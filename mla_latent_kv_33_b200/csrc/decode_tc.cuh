@@ -27,8 +27,9 @@
 //    operands of tile i (one big slot per 64-token block: 256 of this CTA's
 //    latent columns). Every ring item costs a commit (~70 ns of tensor-pipe
 //    time), so items are as large as the shared memory allows. Latent columns
-//    are read twice from L2 (once per operand); HBM sees each cached row
-//    once, brought into L2 by a whole-block prefetch two tiles ahead.
+//    are read twice (once per operand), the second time mostly from L2. (An
+//    explicit whole-block L2 prefetch ahead of the score loads measured
+//    slower: it added DRAM reads without removing the score loads' misses.)
 //  * Loads: a TMA instruction occupies its issuing warp for ~0.3 us whatever
 //    the box size (the lanes of a warp issue in parallel), so three producer
 //    warps share the ring, big slot s belonging to warp s and the small slot
@@ -41,7 +42,9 @@
 //    cut into equal contiguous ranges, one per cluster (persistent grid). A
 //    row whose tiles fall in one range is finished in place (bf16 o_lat,
 //    lse); a row cut by range boundaries leaves normalised fp32 partials
-//    that k_combine merges with a log-sum-exp.
+//    that k_combine merges with a log-sum-exp. (Merging them in the epilogue
+//    of the CTA that finishes a row's last piece measured slower: the merge
+//    then runs on one SM's bandwidth, on that cluster's critical path.)
 //  * Rows past a sequence's end: 64-row blocks wholly past it are loaded at
 //    an out-of-range coordinate (TMA zero fill); the one partially valid block
 //    has its value rows past the end zeroed in shared memory before its PV
@@ -84,7 +87,6 @@ constexpr int MISC_REDL = MISC_RED + 1024;  // float redl[128]
 constexpr int MISC_INTS = MISC_REDL + 512;
 constexpr int MISC_BYTES = MISC_INTS + 64;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-constexpr int PF_TILES = 2;                                // L2 prefetch distance in tiles
 static_assert(NUM_BARS * 8 <= MISC_RED, "barriers overlap the exchange arrays");
 static_assert(SMEM_BYTES <= 232448, "decode shared memory budget");
 static_assert(OFF_P % 1024 == 0 && OFF_BIG % 1024 == 0 && OFF_SMALL % 1024 == 0, "128-byte swizzle alignment");
@@ -103,7 +105,6 @@ __host__ __device__ constexpr int value_item(int i, int n, int v) {
 }
 
 struct Params {
-  const uint8_t *cache;  // base of the cache rows (L2 prefetch addresses)
   const int32_t *seq_lens;
   const int32_t *block_table;
   int64_t max_len;
@@ -150,6 +151,7 @@ struct Piece {
   int bj, t_begin, t_end, vis, nt;
   bool single;
   int slot;
+  int k0, k1;  // clusters holding the first and last piece of the row (slots bj + k0 .. bj + k1)
 };
 
 // Iterates the pieces of this cluster's tile range in order.
@@ -171,7 +173,9 @@ struct PieceIter {
       pc.t_begin = g - off;
       const int e = min(gend, off + nt);
       pc.t_end = e - off;
-      pc.single = (off / Qt) == ((off + nt - 1) / Qt);
+      pc.k0 = off / Qt;
+      pc.k1 = (off + nt - 1) / Qt;
+      pc.single = pc.k0 == pc.k1;
       pc.slot = bj + k;
       g = e;
       off += nt;
@@ -199,7 +203,7 @@ __device__ __forceinline__ void arrive_leader(uint32_t bar_local, uint32_t rank)
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_pf, const __grid_constant__ CUtensorMap tm_v0,
+             const __grid_constant__ CUtensorMap tm_v0,
              const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,7 +248,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_pf);
     tma_prefetch_desc(tm_v);
   }
   if (warp == WARP_MMA) tmem_alloc<2>(smem_u32(tmem_slot), 512);
@@ -332,13 +335,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     // of the slots it owns, so that each slot's uses are issued in order by
     // one warp (a parity wait on the slot's empty barrier is exact only when
     // the waiter is at most one phase ahead). Lane 0 waits for the slot and
-    // arms its full barrier, then lane l issues box l of the item. The L2
-    // prefetch of tile t goes to warp t mod NUM_PRODUCERS.
+    // arms its full barrier, then lane l issues box l of the item.
     const int w = warp;
     const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
     PieceIter it = it0;
     Piece pc;
-    int nbig = 0, nsmall = 0, npc = 0, ntile = 0;
+    int nbig = 0, nsmall = 0, npc = 0;
     bool ok = true;
     auto full_of = [&](int bi) { return rank == 0 ? bar(bi) : mapa_shared(bar(bi), 0); };
     // Next item: 0 if another warp issues it; else waits for its slot, arms
@@ -396,17 +398,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       auto rows_of = [&](int ti, int32_t *r4) {
         for (int v = 0; v < 4; ++v) r4[v] = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * v, pc.vis);
       };
-      auto prefetch = [&](int ti) {  // whole own blocks of tile ti into L2 (lanes 0, 1)
-        if (lane < 2) {
-          const int32_t r = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * (2 * rank + lane), pc.vis);
-          if (r < p.cache_rows) tma_prefetch_3d(&tm_pf, 0, r, 0);
-        }
-        __syncwarp();
-      };
       int32_t cur[4], prev[4], nxt[4];
       rows_of(pc.t_begin, cur);
-      for (int ti = pc.t_begin; ti < min(pc.t_end, pc.t_begin + PF_TILES); ++ti)
-        if (((ntile + ti - pc.t_begin) % NUM_PRODUCERS) == w) prefetch(ti);
       if (w == Q_OWNER) {
         bool good = true;
         if (lane == 0) {
@@ -421,8 +414,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
           break;
         }
       }
-      for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti, ++ntile) {
-        if (ti + PF_TILES < pc.t_end && ((ntile + PF_TILES) % NUM_PRODUCERS) == w) prefetch(ti + PF_TILES);
+      for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti) {
         if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
         const int32_t own[2] = {cur[2 * rank], cur[2 * rank + 1]};
         if (!load_k(own)) { ok = false; break; }
@@ -746,14 +738,14 @@ __global__ void __launch_bounds__(256) k_combine(Params p) {
 
 }  // namespace dec
 
-// Workspace: plan (W, Qt, BJ + 1 offsets) then split partials for at most
+// Workspace: plan (W, Qt, BJ + 1 offsets), then split partials for at most
 // BJ + clusters slots.
+inline size_t decode_plan_bytes(size_t BJ) { return ((BJ + 3) * sizeof(int32_t) + 255) & ~size_t(255); }
 inline size_t decode_tc_ws(int B, int n_q, int sms) {
   const size_t BJ = static_cast<size_t>(B) * n_q;
   const size_t clusters = static_cast<size_t>(sms / 2);
-  const size_t plan = ((BJ + 3) * sizeof(int32_t) + 255) & ~size_t(255);
   const size_t slots = BJ + clusters;
-  return plan + slots * dec::HEADS * dec::DC * sizeof(float) + slots * dec::HEADS * sizeof(float);
+  return decode_plan_bytes(BJ) + slots * dec::HEADS * dec::DC * sizeof(float) + slots * dec::HEADS * sizeof(float);
 }
 
 }  // namespace mla

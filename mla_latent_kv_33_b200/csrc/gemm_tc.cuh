@@ -99,22 +99,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   const CUtensorMap *am = second ? &tm_a2 : &tm_a;
   const int am0 = second ? m0 - p.m_split : m0;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
+    // Lane 0 waits for the stage and arms its barrier; then each box of the
+    // stage is issued by its own lane (a TMA instruction holds its issuing
+    // thread for ~0.3 us, but lanes issue in parallel).
     for (int i = 0; i < nkb; ++i) {
       const int s = i % p.stages;
-      if (i >= p.stages && !mbar_wait(empty(s), ((i / p.stages) - 1) & 1, abort_flag)) break;
-      mbar_arrive_expect_tx(full(s), stage_bytes);
+      bool good = true;
+      if (lane == 0) {
+        if (i >= p.stages) good = mbar_wait(empty(s), ((i / p.stages) - 1) & 1, abort_flag);
+        if (good) mbar_arrive_expect_tx(full(s), stage_bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, good, 0)) break;
       const uint32_t a_dst = sbase + s * stage_bytes;
       const int k0 = (kb0 + i) * BK;
-      if (!p.a_mn_major) {
-        tma_load_2d(a_dst, am, k0, am0 + batch * p.a_batch_rows, full(s));
-      } else {
-        // A(m, k) at W[k][m]: two 64-wide m boxes of 64 k-rows each
-        tma_load_2d(a_dst, am, am0, k0 + batch * p.a_batch_rows, full(s));
+      if (lane == 0) {
+        tma_load_2d(a_dst + A_STAGE, &tm_b, k0 + batch * p.b_batch_cols, n_tile * p.n_tile, full(s));
+      } else if (lane == 1) {
+        if (!p.a_mn_major)
+          tma_load_2d(a_dst, am, k0, am0 + batch * p.a_batch_rows, full(s));
+        else  // A(m, k) at W[k][m]: two 64-wide m boxes of 64 k-rows each
+          tma_load_2d(a_dst, am, am0, k0 + batch * p.a_batch_rows, full(s));
+      } else if (lane == 2 && p.a_mn_major) {
         tma_load_2d(a_dst + A_STAGE / 2, am, am0 + 64, k0 + batch * p.a_batch_rows, full(s));
       }
-      tma_load_2d(a_dst + A_STAGE, &tm_b, k0 + batch * p.b_batch_cols, n_tile * p.n_tile, full(s));
+      __syncwarp();
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -178,9 +188,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             p.dst[static_cast<int64_t>(n) * p.e_split + m] = __float2bfloat16_rn(__uint_as_float(v[c]));
         }
       } else {
-        // q_R rows: lanes (2k, 2k+1) hold the RoPE pair (x[2i], x[2i+1])
+        // q_R rows: lanes (2k, 2k+1) hold the RoPE pair (x[2i], x[2i+1]); the
+        // angle depends on the token only through its position
         const int r = m - p.e_split, h = r / p.d_r, i = r % p.d_r;
         const bool odd = (i & 1) != 0;
+        const double theta = rope_theta(i >> 1, p.d_r, p.rope_base);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int n = n_base + c0 + c;
@@ -188,7 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
           const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
           if (c0 + c < p.n_tile && n < p.n_total) {
             float x0 = odd ? other : mine, x1 = odd ? mine : other;
-            rope_pair(x0, x1, i >> 1, p.d_r, p.positions[n], p.rope_base);
+            rope_rotate(x0, x1, p.positions[n], theta);
             p.q[(static_cast<int64_t>(n) * p.n_h + h) * (p.d_c + p.d_r) + p.d_c + i] = __float2bfloat16_rn(odd ? x1 : x0);
           }
         }
@@ -203,24 +215,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
 // ---------------------------------------------------------- finalizers ----
 
 __device__ __forceinline__ float2 sum_splits2(const float *part, int splits, int64_t stride, int64_t idx) {
-  float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-  int s = 0;
-  for (; s + 4 <= splits; s += 4) {
-    const float2 v0 = *reinterpret_cast<const float2 *>(part + (s + 0) * stride + idx);
-    const float2 v1 = *reinterpret_cast<const float2 *>(part + (s + 1) * stride + idx);
-    const float2 v2 = *reinterpret_cast<const float2 *>(part + (s + 2) * stride + idx);
-    const float2 v3 = *reinterpret_cast<const float2 *>(part + (s + 3) * stride + idx);
-    a.x += v0.x + v1.x;
-    a.y += v0.y + v1.y;
-    b.x += v2.x + v3.x;
-    b.y += v2.y + v3.y;
+  // all loads of a batch of 8 splits are issued before any of them is used
+  float2 acc = make_float2(0.f, 0.f);
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float2 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = s0 + u < splits ? __ldcg(reinterpret_cast<const float2 *>(part + (s0 + u) * stride + idx)) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc.x += v[u].x;
+      acc.y += v[u].y;
+    }
   }
-  for (; s < splits; ++s) {
-    const float2 v = *reinterpret_cast<const float2 *>(part + s * stride + idx);
-    a.x += v.x;
-    a.y += v.y;
-  }
-  return make_float2(a.x + b.x, a.y + b.y);
+  return acc;
 }
 
 // rows [T][576] = sum of splits; RoPE on [512, 576); bf16; store at the

@@ -497,10 +497,9 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   // Views of q and the cache (rows of 576 bf16 = 1152 bytes):
   //   q:        (64 cols, row, 9 chunks of 128 B)        box (64, 64 heads, 9)
   //   score:    (576 cols, row)                          box (64, 64 tokens): one column chunk of a block
-  //   prefetch: (64 cols, row, 9 chunks)                 box (64, 64, 9): a whole block into L2
   //   value:    (64 cols, row, 2 chunks, 2 halves) at column 128 * rank, half stride 256 cols
   //             box (64, 64 tokens, 2, 1) = 128 of this CTA's latent columns of a block
-  CUtensorMap tm_q, tm_k, tm_pf, tm_v[2];
+  CUtensorMap tm_q, tm_k, tm_v[2];
   mla_status s;
   const uint64_t row_b = D::D * 2;
   {
@@ -513,11 +512,6 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
     const uint32_t box[2] = {64, D::BLK};
     if ((s = make_tmap_nd(&tm_k, c->data, 2, dims, str, box, "cache (score chunks)")) != MLA_OK) return s;
   }
-  {
-    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), 9}, str[2] = {row_b, 128};
-    const uint32_t box[3] = {64, D::BLK, 9};
-    if ((s = make_tmap_nd(&tm_pf, c->data, 3, dims, str, box, "cache (block prefetch)")) != MLA_OK) return s;
-  }
   for (int r = 0; r < 2; ++r) {
     const uint64_t dims[4] = {64, static_cast<uint64_t>(rows), 2, 2}, str[3] = {row_b, 128, 512};
     const uint32_t box[4] = {64, D::BLK, 2, 1};
@@ -526,7 +520,6 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   }
 
   D::Params p{};
-  p.cache = static_cast<const uint8_t *>(c->data);
   p.seq_lens = seq_lens;
   p.block_table = c->block_table;
   p.max_len = c->max_len;
@@ -542,7 +535,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.o_lat = static_cast<__nv_bfloat16 *>(o_lat);
   p.lse = lse;
-  const size_t plan_bytes = ((static_cast<size_t>(BJ) + 3) * sizeof(int32_t) + 255) & ~size_t(255);
+  const size_t plan_bytes = mla::decode_plan_bytes(BJ);
   const size_t slots = static_cast<size_t>(BJ) + nclusters;
   p.plan = static_cast<int32_t *>(ws);
   p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan_bytes);
@@ -554,7 +547,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
       return cuda_check("decode: set shared memory size");
     attr_done = true;
   }
-  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k, tm_pf, tm_v[0], tm_v[1], p));
+  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v[0], tm_v[1], p));
   if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
   MLA_LAUNCH(D::k_combine<<<BJ * 16, 256, 0, st>>>(p));
   return cuda_check("decode combine");

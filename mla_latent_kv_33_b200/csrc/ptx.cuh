@@ -186,12 +186,6 @@ __device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int32_t x, int
                : "memory");
 }
 
-__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int32_t x, int32_t y, int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(x), "r"(y),
-               "r"(z)
-               : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 // Shared-memory matrix descriptor, 128-byte swizzle. Addresses/offsets in bytes.
