@@ -32,6 +32,24 @@ METRIC = "MLA decode µs/step, latent-cache HBM GB/s and TFLOP/s vs roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def decode_traffic(workload="v2_b64_paged"):
+    """DRAM bytes of one k_decode launch on the workload, from the committed ncu
+    summary, or None when there is none or the decode source has changed since
+    that capture."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        doc = open(os.path.join(here, "profiles", f"k_decode_{workload}.md")).read()
+        src = open(os.path.join(here, "mla_latent_kv_33_b200", "csrc", "decode_tc.cuh"), "rb").read()
+    except OSError:
+        return None
+    fields = dict(l.split(": ", 1) for l in doc.splitlines() if l.startswith(("traffic_bytes_per_launch:",
+                                                                              "decode_source_sha256_16:")))
+    if fields.get("decode_source_sha256_16", "").strip() != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -384,7 +402,8 @@ def main():
         "peak": peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"],
         "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
         "frac": (t_hbm if bound == "hbm" else t_tc) / dec_s,
-        "traffic": None,
+        "traffic": decode_traffic(w.name),
+        "traffic_kernel": "k_decode (ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch)",
         "peak_source": peak_kind,
         "algorithmic_bytes": work["cache_bytes"], "algorithmic_flops": work["flops"],
         "decode_us": r["dec_ms"] * 1e3,
