@@ -140,6 +140,26 @@ mla_status mla_decode(const mla_dims *dims, const void *q, const mla_cache *cach
                       const int32_t *seq_lens, int32_t B, int32_t n_q, void *o_lat, float *lse,
                       int32_t num_splits, void *ws, size_t ws_bytes, void *stream);
 
+/* mla_decode without a caller workspace. The pages have no counterpart: this
+ * is a convenience of this library for callers that cannot pass scratch
+ * memory. Same computation, arguments (minus num_splits, ws, ws_bytes),
+ * outputs and error behaviour as mla_decode.
+ *   Scratch: a static device array of this library, sized for at most 64 token
+ *   rows (B * n_q <= 64) and 74 decode clusters (one 148-SM B200), about
+ *   35 MB, reserved when the library's device code is loaded. Larger calls
+ *   return MLA_ERR_UNSUPPORTED with the reason in mla_last_error_message().
+ *   The library allocates nothing.
+ *   First call on each device looks up that device's copy of the array
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Nothing in the scratch needs to start at zero: every call writes each
+ *   byte it later reads.
+ *   The scratch is shared by all callers in the process: calls that can
+ *   overlap in time on one device (different streams, or different host
+ *   threads) race on it and must be serialised by the caller. */
+mla_status mla_decode_noalloc(const mla_dims *dims, const void *q, const mla_cache *cache,
+                              const int32_t *seq_lens, int32_t B, int32_t n_q, void *o_lat, float *lse,
+                              void *stream);
+
 /* Per-head readout, decompressed once at the end (MLA walk-through, section
  * 3 order B; DeepSeek-V2 explainer, eq. 11):
  *   o[t][h*d_h + i] = sum_j W_UV[h*d_h + i][j] o_lat[t][h][j].

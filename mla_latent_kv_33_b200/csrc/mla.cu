@@ -18,6 +18,7 @@
 #include <cstring>
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <string>
 
 #include "../../include/mla.h"
@@ -555,6 +556,56 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
 
 }  // namespace
 
+// ------------------------------------------- decode without a caller workspace
+//
+// mla_decode_noalloc runs the same decode as mla_decode, with its scratch in
+// a static device array of this translation unit instead of a caller-provided
+// workspace. The array is sized for at most NOALLOC_MAX_ROWS token rows
+// (B * n_q) and NOALLOC_MAX_CLUSTERS decode clusters (one B200: 148 SMs = 74
+// pairs); larger calls are rejected. Its address is looked up once per device
+// with cudaGetSymbolAddress (first call on that device).
+namespace {
+
+constexpr int32_t NOALLOC_MAX_ROWS = 64;
+constexpr int32_t NOALLOC_MAX_CLUSTERS = 74;
+// plan (rows + 3 ints, 256-byte aligned), then fp32 partials [slots][128][512]
+// and [slots][128] for slots = rows + clusters (the decode workspace layout)
+constexpr size_t NOALLOC_BYTES =
+    ((static_cast<size_t>(NOALLOC_MAX_ROWS) + 3) * sizeof(int32_t) + 255) / 256 * 256 +
+    static_cast<size_t>(NOALLOC_MAX_ROWS + NOALLOC_MAX_CLUSTERS) * mla::dec::HEADS * (mla::dec::DC + 1) * sizeof(float);
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
+
+namespace {
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+
+// Address of this device's copy of g_noalloc_scratch, looked up on the first
+// call from each device.
+mla_status noalloc_scratch(void **ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "mla_decode_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES)
+    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc: device ordinal %d >= %d", dev, NOALLOC_MAX_DEVICES);
+  static std::mutex mu;
+  static void *addr[NOALLOC_MAX_DEVICES] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return fail(MLA_ERR_CUDA, "mla_decode_noalloc: cudaGetSymbolAddress of the scratch: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
 // ------------------------------------------------------------------- C ABI --
 
 extern "C" {
@@ -668,6 +719,23 @@ mla_status mla_decode(const mla_dims *d, const void *q, const mla_cache *c, cons
   }
   if (d->dtype == MLA_BF16) return simt_decode<__nv_bfloat16>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
   return simt_decode<float>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
+}
+
+mla_status mla_decode_noalloc(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens,
+                              int32_t B, int32_t n_q, void *o_lat, float *lse, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (B <= 0 || n_q <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_q must be positive");
+  if (static_cast<int64_t>(B) * n_q > NOALLOC_MAX_ROWS)
+    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc serves at most %d token rows (B * n_q), got %lld",
+                NOALLOC_MAX_ROWS, static_cast<long long>(B) * n_q);
+  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, 0);
+  if (need > NOALLOC_BYTES)
+    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc: this call needs %zu scratch bytes, %zu are reserved", need,
+                NOALLOC_BYTES);
+  void *scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != MLA_OK) return s;
+  return mla_decode(d, q, c, seq_lens, B, n_q, o_lat, lse, 0, scratch, NOALLOC_BYTES, stream);
 }
 
 mla_status mla_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, int32_t T, void *o, void *ws,

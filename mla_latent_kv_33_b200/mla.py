@@ -45,6 +45,7 @@ _lib.mla_absorb_q.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, C.c_int32
 _lib.mla_decode.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P,
                             C.c_int32, _P, _S, _P]
 _lib.mla_out_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
+_lib.mla_decode_noalloc.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P, _P]
 _lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64]
 _lib.mla_workspace_size.restype = C.c_size_t
 _lib.mla_get_device_error.argtypes = [_P]
@@ -54,7 +55,8 @@ _lib.mla_last_error_message.restype = C.c_char_p
 _lib.mla_uses_tensor_cores.argtypes = [C.POINTER(Dims), C.c_int32]
 _lib.mla_uses_tensor_cores.restype = C.c_int32
 _lib.mla_kernel_launches.restype = C.c_uint64
-for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_out_proj", "mla_get_device_error"):
+for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj",
+           "mla_get_device_error"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -144,6 +146,14 @@ def mla_decode(p: Dims, q, cache: Cache, seq_lens, n_q, o_lat, lse=None, num_spl
     _check(_lib.mla_decode(C.byref(p), _ptr(q), C.byref(cache.desc), _ptr(seq_lens), B, n_q,
                            _ptr(o_lat), _ptr(lse), num_splits, _ptr(ws), nbytes, _stream(stream)),
            "mla_decode")
+
+
+def mla_decode_noalloc(p: Dims, q, cache: Cache, seq_lens, n_q, o_lat, lse=None, stream=None):
+    """mla_decode with the library's static scratch (at most 64 token rows; calls
+    that may overlap in time race on the scratch)."""
+    B = seq_lens.shape[0]
+    _check(_lib.mla_decode_noalloc(C.byref(p), _ptr(q), C.byref(cache.desc), _ptr(seq_lens), B, n_q,
+                                   _ptr(o_lat), _ptr(lse), _stream(stream)), "mla_decode_noalloc")
 
 
 def mla_out_proj(p: Dims, o_lat, W_UV, o, ws=None, stream=None):
