@@ -212,6 +212,214 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   if (warp == 1) tmem_dealloc<1>(tmem, tmem_cols);
 }
 
+// ------------------------------------------------ fused per-head absorb ----
+//
+// For one head h (one CTA), T <= 128 token rows:
+//   q_C,h = W_UQ_h c_Q   (128 x T)  -> bf16, kept in shared memory
+//   q_R,h = W_QR_h c_Q   ( 64 x T)  -> RoPE at positions[t] -> q[t][h][d_c + i]
+//   q_lat,h = W_UK_h^T q_C,h (512 x T) -> q[t][h][j]
+// (MLA walk-through, section 1 step 3 and section 3 order B; DeepSeek-V2
+// explainer, eqs. 12-13.) Every CTA streams its head's 192 + 128 weight rows
+// once; q_C never leaves the SM. The q_R product runs as an M = 128 MMA whose
+// upper 64 rows read stale shared memory and are discarded.
+namespace ab {
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB: a 128-row A tile (or two 64 x 64 W_UK^T boxes)
+constexpr int QR_BYTES = 64 * BK * 2;  // 8 KB loaded into a 16 KB slot
+struct Params {
+  int T, n_tile, n_h, d_c, d_r, k_blocks;  // k_blocks = d_cq / 64
+  int stages, stage_bytes, col_stride;      // col_stride: TMEM columns per accumulator
+  __nv_bfloat16 *q;                         // [T][n_h][d_c + d_r]
+  const int32_t *positions;
+  double rope_base;
+};
+__host__ __device__ inline int b2_bytes(int n_tile) { return ((n_tile + 63) / 64) * 128 * 128; }
+inline int stage_bytes(int n_tile) { return 2 * A_BYTES + n_tile * BK * 2; }
+inline int stages(int n_tile) {
+  const int budget = 200 * 1024 - b2_bytes(n_tile);
+  const int s = budget / stage_bytes(n_tile);
+  return s > 8 ? 8 : s;
+}
+inline size_t smem(int n_tile, int st) {
+  return static_cast<size_t>(st) * stage_bytes(n_tile) + b2_bytes(n_tile) + 8 * (2 * st + 3) + 16 + 1024;
+}
+}  // namespace ab
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_absorb_head(const __grid_constant__ CUtensorMap tm_uq, const __grid_constant__ CUtensorMap tm_qr,
+                  const __grid_constant__ CUtensorMap tm_cq, const __grid_constant__ CUtensorMap tm_uk,
+                  const ab::Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.x;
+  const uint32_t b2 = sbase + p.stages * p.stage_bytes;  // q_C,h as the MN-major B of the second product
+  const uint32_t bars = b2 + ab::b2_bytes(p.n_tile);
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
+  const uint32_t p1_done = bars + 8u * (2 * p.stages), b2_full = p1_done + 8, p2_done = p1_done + 16;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.stages * p.stage_bytes + ab::b2_bytes(p.n_tile) +
+                                                     8 * (2 * p.stages + 3));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const int n_p2 = 4 * 2;  // second product: 4 M tiles (512 latent rows) x 2 K blocks (d_h = 128)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(p1_done, 1);
+    mbar_init(b2_full, 4);
+    mbar_init(p2_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc<1>(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    const int total = p.k_blocks + n_p2;
+    int g = 0;
+    for (; g < total; ++g) {
+      const int s = g % p.stages;
+      const bool first = g < p.k_blocks;
+      bool good = true;
+      if (lane == 0) {
+        if (g >= p.stages) good = mbar_wait(empty(s), ((g / p.stages) - 1) & 1, abort_flag);
+        if (good)
+          mbar_arrive_expect_tx(full(s), first ? ab::A_BYTES + ab::QR_BYTES + p.n_tile * BK * 2 : ab::A_BYTES);
+      }
+      if (!__shfl_sync(0xffffffffu, good, 0)) break;
+      const uint32_t st = sbase + s * p.stage_bytes;
+      if (first) {
+        const int k0 = g * BK;
+        if (lane == 0) tma_load_2d(st, &tm_uq, k0, head * BM, full(s));
+        else if (lane == 1) tma_load_2d(st + ab::A_BYTES, &tm_qr, k0, head * p.d_r, full(s));
+        else if (lane == 2) tma_load_2d(st + 2 * ab::A_BYTES, &tm_cq, k0, 0, full(s));
+      } else {
+        // W_UK_h^T tile: latent columns [128 mt + 64 lane, +64) of k rows [64 kb, +64)
+        const int u = g - p.k_blocks, mt = u >> 1, kb = u & 1;
+        if (lane < 2) tma_load_2d(st + lane * (ab::A_BYTES / 2), &tm_uk, BM * mt + 64 * lane, head * BM + 64 * kb, full(s));
+      }
+      __syncwarp();
+    }
+    if (lane == 0)  // drain: the MMA commits to the empty barriers have landed
+      for (int q = g - p.stages; q < g; ++q)
+        if (q >= 0) mbar_wait(empty(q % p.stages), (q / p.stages) & 1, abort_flag);
+  } else if (warp == 1 && lane == 0) {
+    // --------------------------------------------------------- MMA issuer
+    const uint32_t id1 = idesc_bf16(BM, p.n_tile, false, false);
+    const uint32_t id2 = idesc_bf16(BM, p.n_tile, true, true);
+    const uint32_t d1 = tmem, d2 = tmem + p.col_stride;
+    int g = 0;
+    bool ok = true;
+    for (; g < p.k_blocks && ok; ++g) {
+      const int s = g % p.stages;
+      if (!mbar_wait(full(s), (g / p.stages) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t st = sbase + s * p.stage_bytes;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint64_t bd = sdesc_sw128(st + 2 * ab::A_BYTES + kk * 32, 16, 1024);
+        tc_mma<1>(d1, sdesc_sw128(st + kk * 32, 16, 1024), bd, id1, (g > 0 || kk > 0) ? 1u : 0u);
+        tc_mma<1>(d2, sdesc_sw128(st + ab::A_BYTES + kk * 32, 16, 1024), bd, id1, (g > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(empty(s));
+    }
+    tc_commit(p1_done);
+    // second product once q_C,h sits in shared memory (and d1, d2 are drained)
+    if (ok && mbar_wait(b2_full, 0, abort_flag)) {
+      tc_fence_after();
+      for (int u = 0; u < n_p2; ++u, ++g) {
+        const int s = g % p.stages, mt = u >> 1, kb = u & 1;
+        if (!mbar_wait(full(s), (g / p.stages) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t st = sbase + s * p.stage_bytes;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma<1>(tmem + mt * p.col_stride, sdesc_sw128(st + kk * 2048, ab::A_BYTES / 2, 1024),
+                    sdesc_sw128(b2 + kb * 8192 + kk * 2048, 128 * 128, 1024), id2, (kb > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(empty(s));
+      }
+    }
+    tc_commit(p2_done);
+  } else if (warp >= 2) {
+    // ----------------------------------------------------------- epilogue
+    const int sp = warp & 3;
+    const int row = 32 * sp + lane;  // accumulator row of this thread
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
+    const int64_t q_row = static_cast<int64_t>(p.n_h) * (p.d_c + p.d_r);  // q elements per token
+    mbar_wait_warp(p1_done, 0, abort_flag);
+    tc_fence_after();
+    // q_C,h row `row` -> B2 (MN-major, 128-byte swizzle): k = row, n = token
+    for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(lane_addr + c0, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {  // 8 tokens per 16-byte chunk
+        const int t0 = c0 + 8 * ch;
+        if (t0 >= p.n_tile) break;
+        const uint32_t w0 = pack_bf16x2(__uint_as_float(v[8 * ch]), __uint_as_float(v[8 * ch + 1]));
+        const uint32_t w1 = pack_bf16x2(__uint_as_float(v[8 * ch + 2]), __uint_as_float(v[8 * ch + 3]));
+        const uint32_t w2 = pack_bf16x2(__uint_as_float(v[8 * ch + 4]), __uint_as_float(v[8 * ch + 5]));
+        const uint32_t w3 = pack_bf16x2(__uint_as_float(v[8 * ch + 6]), __uint_as_float(v[8 * ch + 7]));
+        const int a = t0 >> 6, c16 = (t0 & 63) >> 3;
+        uint8_t *dst = smem + (b2 - sbase) + a * (128 * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((c16 ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w0, w1, w2, w3);
+      }
+    }
+    // q_R,h rows 0..63 (warps of sub-partitions 0, 1): lanes (2k, 2k+1) hold a RoPE pair
+    if (sp < 2) {
+      const bool odd = (row & 1) != 0;
+      const double theta = rope_theta(row >> 1, p.d_r, p.rope_base);
+      for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + p.col_stride + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int t = c0 + c;
+          const float mine = __uint_as_float(v[c]);
+          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          if (t < p.T) {
+            float x0 = odd ? other : mine, x1 = odd ? mine : other;
+            rope_rotate(x0, x1, p.positions[t], theta);
+            p.q[t * q_row + static_cast<int64_t>(head) * (p.d_c + p.d_r) + p.d_c + row] = __float2bfloat16_rn(odd ? x1 : x0);
+          }
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b2_full);
+    // q_lat,h: rows 128 mt + row of the second product
+    mbar_wait_warp(p2_done, 0, abort_flag);
+    tc_fence_after();
+    for (int mt = 0; mt < 4; ++mt) {
+      const int j = BM * mt + row;
+      for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + mt * p.col_stride + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int t = c0 + c;
+          if (t < p.T) p.q[t * q_row + static_cast<int64_t>(head) * (p.d_c + p.d_r) + j] = __float2bfloat16_rn(__uint_as_float(v[c]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc<1>(tmem, 512);
+}
+
 // ---------------------------------------------------------- finalizers ----
 
 __device__ __forceinline__ float2 sum_splits2(const float *part, int splits, int64_t stride, int64_t idx) {
@@ -282,11 +490,14 @@ inline int n_tile_for(int T) {
   return n < 16 ? 16 : n;
 }
 
-// Pipeline depth: fit two CTAs per SM where the N tile allows (~100 KB each).
-inline int stages_for(int n_tile) {
-  const int budget = 100 * 1024;
+// Pipeline depth: a launch that fits in one wave runs one CTA per SM and may
+// keep ~200 KB of stages in flight; larger launches fit two CTAs per SM
+// (~100 KB each).
+inline int stages_for(int n_tile, int ctas, int sms) {
+  const int budget = (ctas <= sms ? 200 : 100) * 1024;
   int s = budget / (A_STAGE + b_stage_bytes(n_tile));
-  return s > 8 ? 8 : (s < 3 ? 3 : s);
+  const int max_s = ctas <= sms ? 12 : 8;
+  return s > max_s ? max_s : (s < 3 ? 3 : s);
 }
 
 inline size_t smem_for(int n_tile, int stages) {

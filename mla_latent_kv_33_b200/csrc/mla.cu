@@ -330,7 +330,7 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
   p.a_mn_major = a_mn_major ? 1 : 0;
   p.a_batch_rows = a_batch_rows;
   p.b_batch_cols = b_batch_cols;
-  p.stages = G::stages_for(g.n_tile);
+  p.stages = G::stages_for(g.n_tile, g.m_tiles * g.n_tiles * g.batches * g.splits, sm_count());
   const size_t smem = G::smem_for(g.n_tile, p.stages);
   static bool attr = false;
   if (!attr) {
@@ -405,6 +405,36 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   const int64_t pairs = static_cast<int64_t>(T) * d->d_cq / 2;
   MLA_LAUNCH(G::k_fin_store<<<static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256)), 256, 0, st>>>(
       part, a.cq.splits, T, d->d_cq, cq, d->d_cq));
+  if (a.uq.n_tile <= 128) {
+    // one CTA per head: q_C,h = W_UQ_h c_Q, q_R,h = RoPE(W_QR_h c_Q), q_lat,h = W_UK_h^T q_C,h
+    CUtensorMap tq, tr, tc, tk;
+    if ((s = make_tmap_bf16(&tq, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&tr, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 64, "W_QR")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&tc, cq, d->d_cq, T, d->d_cq * 2ull, 64, a.uq.n_tile, "c_Q")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&tk, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UK")) != MLA_OK) return s;
+    G::ab::Params ap{};
+    ap.T = T;
+    ap.n_tile = a.uq.n_tile;
+    ap.n_h = d->n_h;
+    ap.d_c = d->d_c;
+    ap.d_r = d->d_r;
+    ap.k_blocks = d->d_cq / G::BK;
+    ap.stages = G::ab::stages(ap.n_tile);
+    ap.stage_bytes = G::ab::stage_bytes(ap.n_tile);
+    ap.col_stride = (ap.n_tile + 31) / 32 * 32;
+    ap.q = static_cast<__nv_bfloat16 *>(q);
+    ap.positions = positions;
+    ap.rope_base = d->rope_base;
+    const size_t smem = G::ab::smem(ap.n_tile, ap.stages);
+    static bool attr = false;
+    if (!attr) {
+      if (cudaFuncSetAttribute(G::k_absorb_head, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
+        return cuda_check("absorb: set shared memory size");
+      attr = true;
+    }
+    MLA_LAUNCH(G::k_absorb_head<<<d->n_h, G::NUM_THREADS, smem, st>>>(tq, tr, tc, tk, ap));
+    return cuda_check("fused per-head absorb (tensor cores)");
+  }
   // [q_C ; q_R] = [W_UQ ; W_QR] c_Q: q_C to the workspace, q_R rotated into q
   if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&ta2, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK)
