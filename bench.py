@@ -66,6 +66,7 @@ def parse():
     ap.add_argument("--workload", default="v2_b64_paged", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch every call from the host (no CUDA graph)")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0, help="target seconds of oracle work")
     return ap.parse_args()
 
@@ -181,48 +182,82 @@ def run_ours(args, rank, world, local_rank):
     cache = mla.Cache(cache_t, bt)
     p = mla.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base, 0.0, w.dtype)
     T = w.T
-    h = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16).to(dev)
-    pos = torch.from_numpy(x.positions).to(dev)
-    sidx = torch.from_numpy(x.seq_idx).to(dev)
-    sl = torch.from_numpy(x.seq_lens).to(dev)
+    # two sets of the step's input and output buffers, so that the end-to-end
+    # loop can copy the next step's inputs in while this step computes
+    h_host = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16)
+    bufs = [{"h": h_host.to(dev), "pos": torch.from_numpy(x.positions).to(dev),
+             "sidx": torch.from_numpy(x.seq_idx).to(dev), "sl": torch.from_numpy(x.seq_lens).to(dev),
+             "o": torch.empty((T, w.n_h * w.d_h), device=dev, dtype=torch.bfloat16)} for _ in range(2)]
+    o = bufs[0]["o"]
     q = torch.empty((T, w.n_h, w.D), device=dev, dtype=torch.bfloat16)
     o_lat = torch.empty((T, w.n_h, w.d_c), device=dev, dtype=torch.bfloat16)
     lse = torch.empty((T, w.n_h), device=dev, dtype=torch.float32)
-    o = torch.empty((T, w.n_h * w.d_h), device=dev, dtype=torch.bfloat16)
     ws = {op: torch.empty(max(1, mla.workspace_size(p, op, w.B if op == mla.OP_DECODE else T, w.n_q)),
                           dtype=torch.uint8, device=dev)
           for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ)}
-    stream = torch.cuda.current_stream()
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    stream = torch.cuda.Stream(device=dev)  # graph capture needs a non-default stream
+    # the decode is bracketed by timing events in every timed step; "external"
+    # makes them real event-record nodes when the step is captured in a graph
+    ev_dec = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
 
     # the cache append and the query absorption are independent: the append
     # runs on a side stream, joined before the decode reads the cache
     side = torch.cuda.Stream(device=dev)
     ev_fork, ev_join = torch.cuda.Event(), torch.cuda.Event()
 
-    def step(i=None):
+    def step(i=None, b=0):
+        x_ = bufs[b]
         ev_fork.record(stream)
         side.wait_event(ev_fork)
-        mla.mla_cache_append(p, h, W["W_DKV"], W["W_KR"], sidx, pos, cache, ws=ws[mla.OP_APPEND], stream=side)
+        mla.mla_cache_append(p, x_["h"], W["W_DKV"], W["W_KR"], x_["sidx"], x_["pos"], cache,
+                             ws=ws[mla.OP_APPEND], stream=side)
         ev_join.record(side)
-        mla.mla_absorb_q(p, h, W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], pos, q, ws=ws[mla.OP_ABSORB],
-                         stream=stream)
+        mla.mla_absorb_q(p, x_["h"], W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], x_["pos"], q,
+                         ws=ws[mla.OP_ABSORB], stream=stream)
         stream.wait_event(ev_join)
         if i is not None:
             ev_dec[i][0].record(stream)
-        mla.mla_decode(p, q, cache, sl, w.n_q, o_lat, lse, ws=ws[mla.OP_DECODE], stream=stream)
+        mla.mla_decode(p, q, cache, x_["sl"], w.n_q, o_lat, lse, ws=ws[mla.OP_DECODE], stream=stream)
         if i is not None:
             ev_dec[i][1].record(stream)
-        mla.mla_out_proj(p, o_lat, W["W_UV"], o, ws=ws[mla.OP_OUT_PROJ], stream=stream)
+        mla.mla_out_proj(p, o_lat, W["W_UV"], x_["o"], ws=ws[mla.OP_OUT_PROJ], stream=stream)
 
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
 
-    for _ in range(args.warmup):
+    # One eager step first (one-time kernel attributes), then the same C-ABI
+    # calls captured once into CUDA graphs: graph_1[b] holds one step on buffer
+    # set b (warm-up and the end-to-end loop), graph_k the K timed steps.
+    # Replays launch every kernel of the step with no host work between them.
+    with torch.cuda.stream(stream):
         step()
+    torch.cuda.synchronize()
+    graph_1 = graph_k = None
+    launches_k = 0
+    if not args.eager:
+        graph_1, graph_k = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()], torch.cuda.CUDAGraph()
+        for b in range(2):
+            with torch.cuda.graph(graph_1[b], stream=stream):
+                step(b=b)
+        n0 = mla.kernel_launches()
+        with torch.cuda.graph(graph_k, stream=stream):
+            for i in range(args.steps):
+                step(i)
+        launches_k = mla.kernel_launches() - n0  # the kernels graph_k launches per replay
+        torch.cuda.synchronize()
+
+    def one_step(b=0):
+        if graph_1 is not None:
+            graph_1[b].replay()
+        else:
+            step(b=b)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
     torch.cuda.synchronize()
     st = mla.mla_get_device_error(stream)
     if st != mla.MLA_OK:
@@ -233,39 +268,62 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     launches0 = mla.kernel_launches()
-    with ClockSampler(gpu_id_for_smi(torch, local_rank)) as clk:
+    with ClockSampler(gpu_id_for_smi(torch, local_rank)) as clk, torch.cuda.stream(stream):
         h0 = time.perf_counter()
         t0.record(stream)
-        for i in range(args.steps):
-            step(i)
+        if graph_k is not None:
+            graph_k.replay()
+        else:
+            for i in range(args.steps):
+                step(i)
         t1.record(stream)
         torch.cuda.synchronize()
         clk.mark(h0, time.perf_counter())
-    launches = mla.kernel_launches() - launches0
+    launches = mla.kernel_launches() - launches0 + launches_k
     barrier()
     ms_total = t0.elapsed_time(t1)
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
 
-    # end to end through the public API: H2D of the step's inputs from pinned
-    # host memory and D2H of the step's output, inside the timed region
-    h_host = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    pos_host = torch.from_numpy(x.positions).pin_memory()
-    sidx_host = torch.from_numpy(x.seq_idx).pin_memory()
-    sl_host = torch.from_numpy(x.seq_lens).pin_memory()
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    h2d = h_host.numel() * 2 + pos_host.numel() * 4 + sidx_host.numel() * 4 + sl_host.numel() * 4
-    d2h = o_host.numel() * 2
+    # End to end through the public API: every step copies its inputs in from
+    # pinned host memory and its output o back, inside the timed region. The
+    # copies run on their own streams, double-buffered, so that step i + 1's
+    # inputs arrive and step i - 1's output leaves while step i computes
+    # (the way a serving loop overlaps them); e0/e1 bracket all of it.
+    in_host = {"h": h_host.pin_memory(), "pos": torch.from_numpy(x.positions).pin_memory(),
+               "sidx": torch.from_numpy(x.seq_idx).pin_memory(), "sl": torch.from_numpy(x.seq_lens).pin_memory()}
+    o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in in_host.values())
+    d2h = o_host[0].numel() * o_host[0].element_size()
+    h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of set b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # step on set b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # o of set b copied out
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.steps):
-        h.copy_(h_host, non_blocking=True)
-        pos.copy_(pos_host, non_blocking=True)
-        sidx.copy_(sidx_host, non_blocking=True)
-        sl.copy_(sl_host, non_blocking=True)
-        step()
-        o_host.copy_(o, non_blocking=True)
+    h2d_stream.wait_event(e0)
+    d2h_stream.wait_event(e0)
+    for i in range(args.steps):
+        b = i % 2
+        with torch.cuda.stream(h2d_stream):
+            if i >= 2:
+                h2d_stream.wait_event(ev_done[b])  # step i - 2 no longer reads set b
+            for k, t in in_host.items():
+                bufs[b][k].copy_(t, non_blocking=True)
+            ev_in[b].record(h2d_stream)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # o of step i - 2 has left set b
+            one_step(b)
+            ev_done[b].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ev_done[b])
+            o_host[b].copy_(bufs[b]["o"], non_blocking=True)
+            ev_out[b].record(d2h_stream)
+    stream.wait_stream(h2d_stream)
+    stream.wait_stream(d2h_stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -280,7 +338,9 @@ def run_ours(args, rank, world, local_rank):
         tt = torch.tensor([step_ms, dec_ms, e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         step_ms, dec_ms, e2e_ms = (float(v) for v in tt.tolist())
+    del graph_1, graph_k
     return {"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "launch_mode": "eager" if args.eager else "cuda_graph",
             "launches": launches, "clocks": clk.summary(), "x": x, "w": w,
             "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
 
@@ -426,6 +486,10 @@ def main():
         s, sample, cores = oracle_sample(w, x, args.cpu_sample_s)
         line["cpu_baseline"] = {"value": s * 1e6, "unit": "µs/step", "cores": cores, "kind": "oracle",
                                 "sample": sample}
+    line["launch"] = (
+        "eager C-ABI calls" if r["launch_mode"] == "eager" else
+        "the step's four C-ABI calls captured once into a CUDA graph, replayed (timed: one graph of K steps; "
+        "e2e: a one-step graph between the host copies)")
     print(json.dumps(line))
 
 

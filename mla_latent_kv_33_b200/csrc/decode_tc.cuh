@@ -19,22 +19,29 @@
 //  * The 128 x 512 fp32 accumulator O is one whole SM of tensor memory, so it
 //    is split over the pair: 256 columns per CTA, plus two 128-column score
 //    buffers = all 512 columns.
-//  * Shared memory per CTA: Q 72 KB resident per piece, P 32 KB, and a ring
-//    of three 32 KB slots and one 16 KB slot consumed strictly in MMA order:
+//  * Shared memory per CTA: Q 72 KB resident per piece and a ring of four
+//    32 KB slots and one 16 KB slot consumed strictly in MMA order:
 //    the score operands of tile i + 1 (column chunks {0,1} {2,3} {4,5} {6,7}
 //    in big slots, chunk 8 in the small one; each chunk holds this CTA's 128
 //    tokens as 128 rows so that one N = 256 MMA spans them), then the value
-//    operands of tile i (one big slot per 64-token block: 256 of this CTA's
-//    latent columns). Every ring item costs a commit (~70 ns of tensor-pipe
+//    operands of tile i (one big slot per pair of blocks {v, v + 2} and latent
+//    half: 128 of this CTA's latent columns of both). Every ring item costs a commit (~70 ns of tensor-pipe
 //    time), so items are as large as the shared memory allows. Latent columns
 //    are read twice (once per operand), the second time mostly from L2. (An
 //    explicit whole-block L2 prefetch ahead of the score loads measured
 //    slower: it added DRAM reads without removing the score loads' misses.)
 //  * Loads: a TMA instruction occupies its issuing warp for ~0.3 us whatever
 //    the box size (the lanes of a warp issue in parallel), so three producer
-//    warps share the ring, big slot s belonging to warp s and the small slot
-//    and Q to warp 0: every slot's uses are issued in order by one warp, whose
-//    lanes issue an item's boxes together.
+//    warps share the ring, big slot s belonging to warp s mod 3: every slot's
+//    uses are issued in order by one warp, whose lanes issue an item's boxes
+//    together.
+//  * P lives in tensor memory, written by the softmax over the scores it was
+//    made from, as the A operand of PV. A pair MMA with M = 128 reads a row's
+//    16-wide K group from both lane m and lane m + 64 (one copy per half of
+//    N), so each K group pairs 8 tokens of the first CTA's half of the tile
+//    (held by lane m) with 8 of the second's (lane m + 64); the two lanes
+//    trade their halves through shared memory. The value item pairs blocks v
+//    and v + 2 at a fixed 16 KB distance, so that one B descriptor spans both.
 //  * Warp roles: warps 0-2 load, warp 3 of CTA 0 issues the MMAs of the pair,
 //    warps 4-7 of both CTAs run the online softmax (fp32, exp2, O rescaled
 //    only when the running max grows by more than 2^8) and the epilogue.
@@ -61,26 +68,25 @@ constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CT
 // 8 warps = 2 per SM sub-partition, so each thread may hold up to 255 registers
 constexpr int NUM_PRODUCERS = 3, WARP_MMA = 3, WARP_SOFTMAX = 4;
 constexpr int NUM_THREADS = 32 * (WARP_SOFTMAX + 4);
-constexpr int NBIG = NUM_PRODUCERS;  // 32 KB ring slots; big slot s belongs to producer warp s
-constexpr int SMALL_OWNER = 0, Q_OWNER = 0;
+constexpr int NBIG = 4;              // 32 KB ring slots; big slot s belongs to producer warp s % 3
+constexpr int SMALL_OWNER = 1, Q_OWNER = 2;
 constexpr int CHUNK_Q = HPC * 128;   // 64 heads x 64 columns
 constexpr int ATOM = BLK * 128;      // 64 rows x 64 columns (one 128-byte-swizzle atom column)
 constexpr int CHUNK_K = 2 * ATOM;    // one column chunk of the CTA's 128 tokens
 constexpr int BIG = 4 * ATOM, SMALL = 2 * ATOM, HALF = BIG / 2;
-constexpr int K_ITEMS = 5, V_ITEMS = 4;  // per tile: chunks {0,1} {2,3} {4,5} {6,7} {8}; one per block
+constexpr int K_ITEMS = 5, V_ITEMS = 4;  // per tile: chunks {0,1} {2,3} {4,5} {6,7} {8}; (block pair, latent half)
 constexpr int BIG_PER_TILE = 8;          // big-slot uses per tile (4 score + 4 value items)
-constexpr int CHUNK_P = HPC * 128;   // 64 heads x 64 tokens
 constexpr int Q_BYTES = 9 * CHUNK_Q;
-constexpr int P_BYTES = 4 * CHUNK_P;
+constexpr int XBUF_BYTES = 128 * 16 * 4;  // softmax partner exchange: 16 packed P words per thread
 constexpr int OFF_Q = 0;
-constexpr int OFF_P = OFF_Q + Q_BYTES;
-constexpr int OFF_BIG = OFF_P + P_BYTES;
+constexpr int OFF_BIG = OFF_Q + Q_BYTES;
 constexpr int OFF_SMALL = OFF_BIG + NBIG * BIG;
-constexpr int OFF_MISC = OFF_SMALL + SMALL;
+constexpr int OFF_XBUF = OFF_SMALL + SMALL;
+constexpr int OFF_MISC = OFF_XBUF + XBUF_BYTES;
 constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_BIG_FULL = 2, BAR_BIG_EMPTY = BAR_BIG_FULL + NBIG,
               BAR_SMALL_FULL = BAR_BIG_EMPTY + NBIG, BAR_SMALL_EMPTY = BAR_SMALL_FULL + 1,
               BAR_V_LANDED = BAR_SMALL_EMPTY + 1, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
-              BAR_S_FREE = BAR_S_FULL + 2, BAR_P_FULL = BAR_S_FREE + 2, BAR_O_FULL = BAR_P_FULL + 1,
+              BAR_P_FULL = BAR_S_FULL + 2, BAR_O_FULL = BAR_P_FULL + 1,
               BAR_O_FREE = BAR_O_FULL + 1, BAR_EXIT = BAR_O_FREE + 1, NUM_BARS = BAR_EXIT + 1;
 constexpr int MISC_RED = 256;               // float red[2][128]
 constexpr int MISC_REDL = MISC_RED + 1024;  // float redl[128]
@@ -89,9 +95,9 @@ constexpr int MISC_BYTES = MISC_INTS + 64;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(NUM_BARS * 8 <= MISC_RED, "barriers overlap the exchange arrays");
 static_assert(SMEM_BYTES <= 232448, "decode shared memory budget");
-static_assert(OFF_P % 1024 == 0 && OFF_BIG % 1024 == 0 && OFF_SMALL % 1024 == 0, "128-byte swizzle alignment");
+static_assert(OFF_BIG % 1024 == 0 && OFF_SMALL % 1024 == 0, "128-byte swizzle alignment");
 constexpr int MAX_UNITS = (NBIG * BIG + SMALL) / 4 - 1;  // plan scratch aliases the ring
-constexpr int S_COL = 256;                    // TMEM: O at [0,256), scores at [256 + 128 b, +128)
+constexpr int S_COL = 256;  // TMEM: O at [0,256); scores, then P over them, at [256 + 128 b, +128)
 constexpr uint32_t IDESC_S = idesc_bf16(128, 256, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
 constexpr float RESCALE_LOG2 = 8.f;
@@ -99,9 +105,9 @@ constexpr float RESCALE_LOG2 = 8.f;
 // Ring items in MMA consumption order, per piece of n tiles: the score items
 // of tile 0; for every later tile its score items followed by the value items
 // of the tile before it; the value items of the last tile. The big-slot use
-// of the value item (tile i, block v) of a piece:
-__host__ __device__ constexpr int value_item(int i, int n, int v) {
-  return 4 * (i + 2 < n ? i + 2 : n) + 4 * i + v;
+// of the value item (tile i, block pair vp = {vp, vp + 2}, latent half j):
+__host__ __device__ constexpr int value_item(int i, int n, int vp, int j) {
+  return 4 * (i + 2 < n ? i + 2 : n) + 4 * i + 2 * vp + j;
 }
 
 struct Params {
@@ -233,10 +239,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     mbar_init(bar(BAR_SMALL_EMPTY), 1);
     mbar_init(bar(BAR_V_LANDED), 1);
     mbar_init(bar(BAR_ZERO_DONE), 8);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(BAR_S_FULL + b), 1);
-      mbar_init(bar(BAR_S_FREE + b), 8);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(bar(BAR_S_FULL + b), 1);
     mbar_init(bar(BAR_P_FULL), 8);
     mbar_init(bar(BAR_O_FULL), 1);
     mbar_init(bar(BAR_O_FREE), 8);
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         slot = 0;
         use = nsmall++;
       }
-      if ((big ? slot : SMALL_OWNER) != w) return 0;
+      if ((big ? slot % NUM_PRODUCERS : SMALL_OWNER) != w) return 0;
       const int eb = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
       *fb = big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL;
       bool good = true;
@@ -381,16 +384,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       }
       return true;
     };
-    auto load_v = [&](const int32_t *rows) -> bool {  // value items of one tile: block v, both latent halves
-      for (int v = 0; v < 4; ++v) {
-        int fb = 0;
-        const int off = claim(true, BIG, &fb);
-        if (off < 0) return false;
-        if (off == 0) continue;
-        if (lane < 2)  // lane j: latent half j (16 KB)
-          tma_load_4d_pair(sbase + off + lane * HALF, tm_v, 0, rows[v], 0, lane, full_of(fb));
-        __syncwarp();
-      }
+    // value items of one tile: (block pair {vp, vp + 2}, latent half j); lane l
+    // loads block vp + 2 l (16 KB: two latent chunks of 64 rows)
+    auto load_v = [&](const int32_t *rows) -> bool {
+      for (int vp = 0; vp < 2; ++vp)
+        for (int j = 0; j < 2; ++j) {
+          int fb = 0;
+          const int off = claim(true, BIG, &fb);
+          if (off < 0) return false;
+          if (off == 0) continue;
+          if (lane < 2) tma_load_4d_pair(sbase + off + lane * HALF, tm_v, 0, rows[vp + 2 * lane], 0, j, full_of(fb));
+          __syncwarp();
+        }
       return true;
     };
     while (ok && it.next(p, pc)) {
@@ -430,8 +435,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     // drain: every commit aimed at the empty barriers of this warp's slots
     // (and of Q) has landed; each warp waits only on what it owns, see above
     if (lane == 0) {
-      const int uses = nbig > w ? (nbig - w + NBIG - 1) / NBIG : 0;
-      if (ok && uses > 0) mbar_wait(bar(BAR_BIG_EMPTY + w), (uses - 1) & 1, abort_flag);
+      for (int sl = w; ok && sl < NBIG; sl += NUM_PRODUCERS) {
+        const int uses = nbig > sl ? (nbig - sl + NBIG - 1) / NBIG : 0;
+        if (uses > 0) mbar_wait(bar(BAR_BIG_EMPTY + sl), (uses - 1) & 1, abort_flag);
+      }
       if (ok && w == SMALL_OWNER && nsmall > 0) mbar_wait(bar(BAR_SMALL_EMPTY), (nsmall - 1) & 1, abort_flag);
       if (ok && w == Q_OWNER && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
     }
@@ -458,32 +465,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         return sbase + (big ? OFF_BIG + slot * BIG : OFF_SMALL);
       };
       auto release = [&]() { tc_commit_pair(bar(empty_bar), 0x3); };
-      // PV of global tile gt (tile ti of the current piece)
+      // PV of global tile gt (tile ti of the current piece): A = P in tensor
+      // memory; K step m of value item (vp, j) takes 8 tokens of block vp and 8
+      // of block vp + 2 (one B descriptor over both halves of the item)
       auto issue_pv = [&](int gt, int ti, bool first) -> bool {
         const int zc = partial_chunk(pc.vis, ti);
-        for (int v = 0; v < 4; ++v) {
-          const uint32_t vb = take(true);
-          if (vb == 0) return false;
-          if (v == 0) {
-            if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
-            if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
-          }
-          if (v == zc) {  // both CTAs zero the rows past the end of this slab first
-            mbar_arrive(bar(BAR_V_LANDED));
-            mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
-            if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
-            ++gz;
-            tc_fence_after();
-          }
-          const uint32_t pa = sbase + OFF_P + v * CHUNK_P;
+        const uint32_t p_col = tmem + S_COL + 128 * (gt & 1);
+        for (int vp = 0; vp < 2; ++vp)
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t vb = take(true);
+            if (vb == 0) return false;
+            if (vp == 0 && j == 0) {
+              if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
+              if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+              tc_fence_after();
+            }
+            if (zc >= 0 && vp == (zc & 1)) {  // both CTAs zero the rows past the end first
+              mbar_arrive(bar(BAR_V_LANDED));
+              mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
+              if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
+              ++gz;
+              tc_fence_after();
+            }
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              tc_mma<2>(tmem + 128 * j, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(vb + j * HALF + kk * 2048, ATOM, 1024),
-                        IDESC_PV, (first && v == 0 && kk == 0) ? 0u : 1u);
-          release();
-        }
+            for (int m = 0; m < 8; ++m)
+              tc_mma_ts<2>(tmem + 128 * j, p_col + 8 * (8 * vp + m), sdesc_sw128(vb + m * 1024, ATOM, HALF), IDESC_PV,
+                           (first && vp == 0 && m == 0) ? 0u : 1u);
+            release();
+          }
         tc_commit_pair(bar(BAR_O_FULL), 0x3);
         return true;
       };
@@ -491,8 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         if (!mbar_wait(bar(BAR_Q_FULL), npc & 1, abort_flag)) break;
         const int n = pc.t_end - pc.t_begin;
         for (int i = 0; i < n && ok; ++i, ++gi) {
-          const int b = gi & 1;
-          if (gi >= 2 && !mbar_wait(bar(BAR_S_FREE + b), ((gi >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          const int b = gi & 1;  // S(gi) goes over P(gi - 2), read by PV(gi - 2), issued before it
           for (int q = 0; q < K_ITEMS; ++q) {
             const bool big = q < K_ITEMS - 1;
             const uint32_t kbuf = take(big);
@@ -566,28 +574,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
             m_ref = mx;
           }
         }
-        // pass 2: p = exp2((s - m) * scale * log2 e), packed to bf16 in registers
+        // pass 2: p = exp2((s - m) * scale * log2 e) as bf16 pairs. Chunk q4 holds
+        // K groups 4 q4 .. 4 q4 + 3; a group is 8 tokens of each half of the tile,
+        // the first half in columns 8 g + 0..3 and the second in 8 g + 4..7, in
+        // both lanes of the row. The partner lane (L ^ 64) holds the other half.
         const float mo = m_ref * c2;
-        uint32_t pk[64];
         float ps = 0.f;
-#pragma unroll
+        uint4 *xb = reinterpret_cast<uint4 *>(smem + OFF_XBUF);
+#pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t sr[32];
           tmem_ld32(s_addr + 32 * q4, sr);
           tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int t = tok0 + 32 * q4 + 2 * c;
             const float p0 = t < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c]), c2, -mo)) : 0.f;
             const float p1 = t + 1 < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), c2, -mo)) : 0.f;
             ps += p0 + p1;
-            pk[16 * q4 + c] = pack_bf16x2(p0, p1);
+            pk[c] = pack_bf16x2(p0, p1);
           }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) xb[L * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          named_bar_sync(1, 128);
+          uint32_t pw[32];
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const uint4 o = xb[(L ^ 64) * 4 + gg];
+            const uint32_t mine[4] = {pk[4 * gg], pk[4 * gg + 1], pk[4 * gg + 2], pk[4 * gg + 3]};
+            const uint32_t theirs[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              pw[8 * gg + e] = half == 0 ? mine[e] : theirs[e];
+              pw[8 * gg + 4 + e] = half == 0 ? theirs[e] : mine[e];
+            }
+          }
+          tmem_st32(s_addr + 32 * q4, pw);
+          named_bar_sync(1, 128);  // the exchange buffer is reused by the next chunk
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_leader(bar(BAR_S_FREE + b), rank);
-        // the single P buffer and O are free once the previous tile's PV is done
+        tmem_wait_st();
+        // O is rescaled only after the previous tile's PV has finished with it
         if (gi > 0) mbar_wait_warp(bar(BAR_O_FULL), (gi - 1) & 1, abort_flag);
         tc_fence_after();
         if (rescale) {
@@ -604,34 +631,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
           tmem_wait_st();
         }
         lsum = lsum * alpha + ps;
-        // P: row `row`, tokens tok0 .. tok0 + 127 -> chunks 2*half, 2*half + 1 (SW128, K-major)
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int chunk = 2 * half + (u >> 3), w16 = u & 7;
-          uint8_t *dst = smem + OFF_P + chunk * CHUNK_P + row * 128 + ((w16 ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_leader(bar(BAR_P_FULL), rank);
-        // partial block of the last tile: zero its value rows past the end
-        // (the MMA thread signals when that slab has landed)
+        // partial block of the last tile: zero its value rows past the end in
+        // the two value items (latent halves) that hold it; the MMA thread
+        // signals as each one lands
         const int zc = partial_chunk(pc.vis, ti);
         if (zc >= 0) {
           const int valid = vis_t - BLK * zc;
           const int nrow = BLK - valid;
-          mbar_wait_warp(bar(BAR_V_LANDED), gz & 1, abort_flag);
-          ++gz;
-          uint8_t *vb = smem + OFF_BIG + ((bbase + value_item(i, n, zc)) % NBIG) * BIG;
-          // slab = [latent half j][chunk a][64 rows][128 B]: 32 16-byte words per row
-          for (int e = L; e < nrow * 32; e += 128) {
-            const int r = valid + e / 32, j = (e >> 4) & 1, a = (e >> 3) & 1, w16 = e & 7;
-            *reinterpret_cast<uint4 *>(vb + j * HALF + a * ATOM + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
+          for (int j = 0; j < 2; ++j) {
+            mbar_wait_warp(bar(BAR_V_LANDED), gz & 1, abort_flag);
+            ++gz;
+            uint8_t *vb = smem + OFF_BIG + ((bbase + value_item(i, n, zc & 1, j)) % NBIG) * BIG + (zc >> 1) * HALF;
+            // block slab = [chunk a][64 rows][128 B]: 16 16-byte words per row
+            for (int e = L; e < nrow * 16; e += 128) {
+              const int r = valid + e / 16, a = (e >> 3) & 1, w16 = e & 7;
+              *reinterpret_cast<uint4 *>(vb + a * ATOM + r * 128 + w16 * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) arrive_leader(bar(BAR_ZERO_DONE), rank);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) arrive_leader(bar(BAR_ZERO_DONE), rank);
         }
       }
       // ---------------------------------------------------------- epilogue
@@ -696,42 +718,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
 
 // Merge the split partials of every token row that was cut by cluster range
 // boundaries: lse = log sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s.
-// grid = BJ * 16 blocks of 8 warps; one warp per head.
-__global__ void __launch_bounds__(256) k_combine(Params p) {
-  const int bj = blockIdx.x >> 4, head = (blockIdx.x & 15) * 8 + (threadIdx.x >> 5);
+// grid = BJ * 32 blocks of 128 threads: warp w of block g handles head
+// 4 (g mod 32) + w of row g / 32, lane l its float4 columns l + 32 c, c < 4.
+// The partials of COMBINE_CHUNK pieces (their lse and all four float4) are
+// loaded together, one round trip per chunk, and merged with a running max.
+constexpr int COMBINE_CHUNK = 2, COMBINE_BLOCKS_PER_ROW = HEADS / 4;
+__global__ void __launch_bounds__(128) k_combine(Params p) {
+  const int bj = blockIdx.x / COMBINE_BLOCKS_PER_ROW;
+  const int head = 4 * (blockIdx.x % COMBINE_BLOCKS_PER_ROW) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int a = p.plan[2 + bj], e = p.plan[3 + bj], Qt = p.plan[1];
   if (e <= a) return;
   const int k0 = a / Qt, k1 = (e - 1) / Qt;
   if (k0 == k1) return;
-  float M = -INFINITY;
-  for (int k = k0; k <= k1; ++k) M = fmaxf(M, p.part_lse[static_cast<int64_t>(bj + k) * HEADS + head]);
-  float Z = 0.f;
-  float acc[16];
+  const int np = k1 - k0 + 1;
+  const float *pl = p.part_lse + static_cast<int64_t>(bj + k0) * HEADS + head;
+  const float4 *po =
+      reinterpret_cast<const float4 *>(p.part_o + (static_cast<int64_t>(bj + k0) * HEADS + head) * DC) + lane;
+  constexpr int64_t PIECE4 = static_cast<int64_t>(HEADS) * DC / 4;  // float4 stride between pieces
+  float M = -INFINITY, Z = 0.f;
+  float4 acc[4];
 #pragma unroll
-  for (int v = 0; v < 16; ++v) acc[v] = 0.f;
-  for (int k = k0; k <= k1; ++k) {
-    const float w = __expf(p.part_lse[static_cast<int64_t>(bj + k) * HEADS + head] - M);
-    Z += w;
-    const float4 *src = reinterpret_cast<const float4 *>(p.part_o + (static_cast<int64_t>(bj + k) * HEADS + head) * DC);
+  for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < np; k += COMBINE_CHUNK) {
+    float l[COMBINE_CHUNK];
+    float4 x[COMBINE_CHUNK][4];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const float4 x = src[lane + 32 * v];
-      acc[4 * v] += w * x.x;
-      acc[4 * v + 1] += w * x.y;
-      acc[4 * v + 2] += w * x.z;
-      acc[4 * v + 3] += w * x.w;
+    for (int u = 0; u < COMBINE_CHUNK; ++u) {
+      if (k + u < np) {
+        l[u] = __ldcg(pl + static_cast<int64_t>(k + u) * HEADS);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) x[u][c] = __ldcg(po + (k + u) * PIECE4 + 32 * c);
+      } else {
+        l[u] = -INFINITY;
+      }
     }
+    float Mn = M;
+#pragma unroll
+    for (int u = 0; u < COMBINE_CHUNK; ++u) Mn = fmaxf(Mn, l[u]);
+    const float r = __expf(M - Mn);  // 0 on the first chunk (M = -inf, Mn finite)
+    Z *= r;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      acc[c].x *= r;
+      acc[c].y *= r;
+      acc[c].z *= r;
+      acc[c].w *= r;
+    }
+#pragma unroll
+    for (int u = 0; u < COMBINE_CHUNK; ++u) {
+      if (k + u < np) {
+        const float wgt = __expf(l[u] - Mn);
+        Z += wgt;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[c].x += wgt * x[u][c].x;
+          acc[c].y += wgt * x[u][c].y;
+          acc[c].z += wgt * x[u][c].z;
+          acc[c].w += wgt * x[u][c].w;
+        }
+      }
+    }
+    M = Mn;
   }
   const float inv = 1.f / Z;
-  __nv_bfloat16 *dst = p.o_lat + (static_cast<int64_t>(bj) * HEADS + head) * DC;
+  uint2 *dst = reinterpret_cast<uint2 *>(p.o_lat + (static_cast<int64_t>(bj) * HEADS + head) * DC) + lane;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    const int col = 4 * (lane + 32 * v);
-    uint2 w;
-    w.x = pack_bf16x2(acc[4 * v] * inv, acc[4 * v + 1] * inv);
-    w.y = pack_bf16x2(acc[4 * v + 2] * inv, acc[4 * v + 3] * inv);
-    *reinterpret_cast<uint2 *>(dst + col) = w;
+  for (int c = 0; c < 4; ++c) {
+    uint2 out;
+    out.x = pack_bf16x2(acc[c].x * inv, acc[c].y * inv);
+    out.y = pack_bf16x2(acc[c].z * inv, acc[c].w * inv);
+    dst[32 * c] = out;
   }
   if (lane == 0 && p.lse != nullptr) p.lse[static_cast<int64_t>(bj) * HEADS + head] = M + logf(Z);
 }

@@ -580,7 +580,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   }
   MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v[0], tm_v[1], p));
   if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
-  MLA_LAUNCH(D::k_combine<<<BJ * 16, 256, 0, st>>>(p));
+  MLA_LAUNCH(D::k_combine<<<BJ * D::COMBINE_BLOCKS_PER_ROW, 128, 0, st>>>(p));
   return cuda_check("decode combine");
 }
 
