@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every call from the host (no CUDA graph)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch kernels without programmatic dependent launch (mla_set_launch_overlap off)")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0, help="target seconds of oracle work")
     return ap.parse_args()
 
@@ -228,6 +230,10 @@ def run_ours(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
+    # launch overlap: each tensor-core kernel may be scheduled, set up and
+    # start streaming its weights while the kernel ahead of it finishes
+    mla.set_launch_overlap(not args.no_overlap)
+
     # One eager step first (one-time kernel attributes), then the same C-ABI
     # calls captured once into CUDA graphs: graph_1[b] holds one step on buffer
     # set b (warm-up and the end-to-end loop), graph_k the K timed steps.
@@ -340,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
         step_ms, dec_ms, e2e_ms = (float(v) for v in tt.tolist())
     del graph_1, graph_k
     return {"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launch_mode": "eager" if args.eager else "cuda_graph",
+            "launch_mode": ("eager" if args.eager else "cuda_graph") + ("" if args.no_overlap else "+overlap"),
             "launches": launches, "clocks": clk.summary(), "x": x, "w": w,
             "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
 
@@ -487,9 +493,10 @@ def main():
         line["cpu_baseline"] = {"value": s * 1e6, "unit": "µs/step", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     line["launch"] = (
-        "eager C-ABI calls" if r["launch_mode"] == "eager" else
-        "the step's four C-ABI calls captured once into a CUDA graph, replayed (timed: one graph of K steps; "
-        "e2e: a one-step graph between the host copies)")
+        ("eager C-ABI calls" if r["launch_mode"].startswith("eager") else
+         "the step's four C-ABI calls captured once into a CUDA graph, replayed (timed: one graph of K steps; "
+         "e2e: a one-step graph between the host copies)")
+        + ("; launch overlap on (programmatic dependent launch)" if r["launch_mode"].endswith("+overlap") else ""))
     print(json.dumps(line))
 
 

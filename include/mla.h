@@ -188,6 +188,19 @@ const char *mla_last_error_message(void);
  * tensor-core kernels are not built for). */
 int32_t mla_uses_tensor_cores(const mla_dims *dims, int32_t op);
 
+/* Launch overlap (process-wide, off by default). When on, every tensor-core
+ * kernel is launched with programmatic stream serialization: it may be
+ * scheduled while the kernel ahead of it on the stream is still running, set
+ * up its barriers and tensor memory, and start streaming the weight matrices
+ * of its call (W_DKV/W_KR, W_DQ, W_UQ/W_QR/W_UK, W_UV); it reads activations,
+ * the cache, sequence lengths or positions, and writes any output, only
+ * after that kernel has completed. The caller guarantees that the weights of
+ * a call are not written by the work enqueued on the stream just before it.
+ * Results are identical either way. Returns MLA_OK. No counterpart on the
+ * pages: it is a property of how the calls are launched, not of the method. */
+mla_status mla_set_launch_overlap(int32_t enable);
+int32_t mla_get_launch_overlap(void);
+
 /* Number of kernels this library has launched in this process (all devices,
  * all threads). Lets callers count launches inside a timed region. */
 uint64_t mla_kernel_launches(void);

@@ -142,15 +142,31 @@ __device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out)
 // First cache row of the 64-row block at token `pos` of sequence b, or
 // p.cache_rows (out of range: the TMA load zero-fills) when the block lies
 // past `vis` or its block-table entry is invalid.
-__device__ __forceinline__ int32_t block_row(const Params &p, int b, int64_t pos, int vis) {
-  if (pos >= vis) return static_cast<int32_t>(p.cache_rows);
-  if (!p.paged) return static_cast<int32_t>(static_cast<int64_t>(b) * p.max_len + pos);
-  const int32_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + pos / p.block_size];
-  if (blk < 0 || blk >= p.num_blocks_i32) {
-    dev_error(MLA_DEVERR_DATA);
-    return static_cast<int32_t>(p.cache_rows);
+// Cache rows of the four 64-token blocks of a 256-token tile (positions
+// t0 + 64 v), or cache_rows (an out-of-range TMA coordinate: zero fill) for
+// blocks past the visible length. The four block-table entries are loaded
+// before any of them is checked, so that their latencies overlap.
+__device__ __forceinline__ void tile_rows(const Params &p, int b, int64_t t0, int vis, int32_t r4[4]) {
+  int32_t blk[4];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int64_t pos = t0 + BLK * v;
+    blk[v] = p.paged && pos < vis ? p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + pos / p.block_size] : 0;
   }
-  return static_cast<int32_t>(static_cast<int64_t>(blk) * p.block_size + pos % p.block_size);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int64_t pos = t0 + BLK * v;
+    if (pos >= vis) {
+      r4[v] = static_cast<int32_t>(p.cache_rows);
+    } else if (!p.paged) {
+      r4[v] = static_cast<int32_t>(static_cast<int64_t>(b) * p.max_len + pos);
+    } else if (blk[v] < 0 || blk[v] >= p.num_blocks_i32) {
+      dev_error(MLA_DEVERR_DATA);
+      r4[v] = static_cast<int32_t>(p.cache_rows);
+    } else {
+      r4[v] = static_cast<int32_t>(static_cast<int64_t>(blk[v]) * p.block_size + pos % p.block_size);
+    }
+  }
 }
 
 struct Piece {
@@ -254,6 +270,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     tma_prefetch_desc(tm_v);
   }
   if (warp == WARP_MMA) tmem_alloc<2>(smem_u32(tmem_slot), 512);
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  // everything below reads sequence lengths, the cache or q, or writes the
+  // workspace: only once the previous kernel on the stream has finished
+  griddep_wait();
 
   // ---- plan: tiles per unit, prefix sums, this cluster's first unit ----
   const int BJ = p.B * p.n_q;
@@ -393,17 +413,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
           const int off = claim(true, BIG, &fb);
           if (off < 0) return false;
           if (off == 0) continue;
-          if (lane < 2) tma_load_4d_pair(sbase + off + lane * HALF, tm_v, 0, rows[vp + 2 * lane], 0, j, full_of(fb));
+          const int32_t row = lane ? (vp ? rows[3] : rows[2]) : (vp ? rows[1] : rows[0]);  // block vp + 2 lane
+          if (lane < 2) tma_load_4d_pair(sbase + off + lane * HALF, tm_v, 0, row, 0, j, full_of(fb));
           __syncwarp();
         }
       return true;
     };
     while (ok && it.next(p, pc)) {
       const int b = pc.bj / p.n_q;
-      auto rows_of = [&](int ti, int32_t *r4) {
-        for (int v = 0; v < 4; ++v) r4[v] = block_row(p, b, static_cast<int64_t>(ti) * TILE + BLK * v, pc.vis);
-      };
-      int32_t cur[4], prev[4], nxt[4];
+      auto rows_of = [&](int ti, int32_t *r4) { tile_rows(p, b, static_cast<int64_t>(ti) * TILE, pc.vis, r4); };
+      int32_t cur[4], prev[4], nxt[4] = {0, 0, 0, 0};
       rows_of(pc.t_begin, cur);
       if (w == Q_OWNER) {
         bool good = true;
@@ -421,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       }
       for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti) {
         if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
-        const int32_t own[2] = {cur[2 * rank], cur[2 * rank + 1]};
+        const int32_t own[2] = {rank ? cur[2] : cur[0], rank ? cur[3] : cur[1]};
         if (!load_k(own)) { ok = false; break; }
         if (ti > pc.t_begin && !load_v(prev)) { ok = false; break; }
         for (int v = 0; v < 4; ++v) {
@@ -724,6 +743,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
 // loaded together, one round trip per chunk, and merged with a running max.
 constexpr int COMBINE_CHUNK = 2, COMBINE_BLOCKS_PER_ROW = HEADS / 4;
 __global__ void __launch_bounds__(128) k_combine(Params p) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
   const int bj = blockIdx.x / COMBINE_BLOCKS_PER_ROW;
   const int head = 4 * (blockIdx.x % COMBINE_BLOCKS_PER_ROW) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;

@@ -50,6 +50,7 @@ struct Params {
   int n_h, d_c, d_r;
   double rope_base;
   const int32_t *positions;
+  int prefetch;  // launched with launch overlap: weight boxes of the first stages go out before griddep_wait
 };
 
 __host__ __device__ constexpr int b_stage_bytes(int n_tile) { return n_tile * BK * 2; }
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   const int m0 = m_tile * BM;
   const bool second = m0 >= p.m_split;
@@ -101,10 +103,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
-    // Lane 0 waits for the stage and arms its barrier; then each box of the
-    // stage is issued by its own lane (a TMA instruction holds its issuing
-    // thread for ~0.3 us, but lanes issue in parallel).
-    for (int i = 0; i < nkb; ++i) {
+    // A TMA instruction holds its issuing thread for ~0.3 us, but lanes issue
+    // in parallel, so every box goes out from its own lane. Under launch
+    // overlap the first stages are armed together and their weight boxes
+    // issued before the wait for the previous kernel on the stream (weights
+    // do not depend on it), their token boxes after it. Otherwise the stages
+    // go out in order, each stage's boxes together, so that the first stage
+    // is not queued behind the weights of all the others.
+    const uint32_t stage0 = sbase;
+    auto issue_a = [&](int i, int box) {  // box 1: second 64-wide m box of an MN-major A
+      const uint32_t a_dst = stage0 + (i % p.stages) * stage_bytes;
+      const int k0 = (kb0 + i) * BK;
+      if (!p.a_mn_major)
+        tma_load_2d(a_dst, am, k0, am0 + batch * p.a_batch_rows, full(i % p.stages));
+      else  // A(m, k) at W[k][m]: two 64-wide m boxes of 64 k-rows each
+        tma_load_2d(a_dst + box * (A_STAGE / 2), am, am0 + 64 * box, k0 + batch * p.a_batch_rows, full(i % p.stages));
+    };
+    auto issue_b = [&](int i) {
+      const uint32_t a_dst = stage0 + (i % p.stages) * stage_bytes;
+      tma_load_2d(a_dst + A_STAGE, &tm_b, (kb0 + i) * BK + batch * p.b_batch_cols, n_tile * p.n_tile, full(i % p.stages));
+    };
+    const int pre = p.prefetch ? min(nkb, p.stages) : 0;  // stages <= 12: lanes l and 16 + l serve stage l
+    if (lane == 0)
+      for (int i = 0; i < pre; ++i) mbar_arrive_expect_tx(full(i), stage_bytes);
+    __syncwarp();
+    if (lane < pre) issue_a(lane, 0);
+    else if (lane >= 16 && lane - 16 < pre && p.a_mn_major) issue_a(lane - 16, 1);
+    griddep_wait();
+    if (lane < pre) issue_b(lane);
+    __syncwarp();
+    for (int i = pre; i < nkb; ++i) {
       const int s = i % p.stages;
       bool good = true;
       if (lane == 0) {
@@ -112,18 +140,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         if (good) mbar_arrive_expect_tx(full(s), stage_bytes);
       }
       if (!__shfl_sync(0xffffffffu, good, 0)) break;
-      const uint32_t a_dst = sbase + s * stage_bytes;
-      const int k0 = (kb0 + i) * BK;
-      if (lane == 0) {
-        tma_load_2d(a_dst + A_STAGE, &tm_b, k0 + batch * p.b_batch_cols, n_tile * p.n_tile, full(s));
-      } else if (lane == 1) {
-        if (!p.a_mn_major)
-          tma_load_2d(a_dst, am, k0, am0 + batch * p.a_batch_rows, full(s));
-        else  // A(m, k) at W[k][m]: two 64-wide m boxes of 64 k-rows each
-          tma_load_2d(a_dst, am, am0, k0 + batch * p.a_batch_rows, full(s));
-      } else if (lane == 2 && p.a_mn_major) {
-        tma_load_2d(a_dst + A_STAGE / 2, am, am0 + 64, k0 + batch * p.a_batch_rows, full(s));
-      }
+      if (lane == 0) issue_b(i);
+      else if (lane == 1) issue_a(i, 0);
+      else if (lane == 2 && p.a_mn_major) issue_a(i, 1);
       __syncwarp();
     }
   } else if (warp == 1 && lane == 0) {
@@ -149,6 +168,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     // ------------------------------------------------------------- epilogue
     const int sp = warp & 3;
     const int row = 32 * sp + lane;  // m within tile
+    griddep_wait();  // outputs are written only once the previous kernel has finished
     mbar_wait_warp(done, 0, abort_flag);
     tc_fence_after();
     const int m = m0 + row;
@@ -231,6 +251,7 @@ struct Params {
   __nv_bfloat16 *q;                         // [T][n_h][d_c + d_r]
   const int32_t *positions;
   double rope_base;
+  int prefetch;  // launched with launch overlap: weight boxes of the first stages go out before griddep_wait
 };
 __host__ __device__ inline int b2_bytes(int n_tile) { return ((n_tile + 63) / 64) * 128 * 128; }
 inline int stage_bytes(int n_tile) { return 2 * A_BYTES + n_tile * BK * 2; }
@@ -279,32 +300,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
+    // Under launch overlap the first stages are armed together and their
+    // weight boxes issued by lanes l (W_UQ or W_UK box 0) and 8 + l (W_QR or
+    // W_UK box 1) before the wait for the previous kernel on the stream;
+    // their c_Q boxes (lane l) only after it. Every other stage, in order:
+    // lane 0 waits and arms, lanes 0-2 issue.
     const int total = p.k_blocks + n_p2;
-    int g = 0;
+    const int pre = p.prefetch ? min(total, p.stages) : 0;  // stages <= 8
+    auto stage_tx = [&](int g) { return g < p.k_blocks ? ab::A_BYTES + ab::QR_BYTES + p.n_tile * BK * 2 : ab::A_BYTES; };
+    auto issue_w = [&](int g, int box) {  // weight box `box` (0, 1) of item g
+      const int s = g % p.stages;
+      const uint32_t st = sbase + s * p.stage_bytes;
+      if (g < p.k_blocks) {
+        if (box == 0) tma_load_2d(st, &tm_uq, g * BK, head * BM, full(s));
+        else tma_load_2d(st + ab::A_BYTES, &tm_qr, g * BK, head * p.d_r, full(s));
+      } else {
+        // W_UK_h^T tile: latent columns [128 mt + 64 box, +64) of k rows [64 kb, +64)
+        const int u = g - p.k_blocks, mt = u >> 1, kb = u & 1;
+        tma_load_2d(st + box * (ab::A_BYTES / 2), &tm_uk, BM * mt + 64 * box, head * BM + 64 * kb, full(s));
+      }
+    };
+    auto issue_cq = [&](int g) {
+      const int s = g % p.stages;
+      tma_load_2d(sbase + s * p.stage_bytes + 2 * ab::A_BYTES, &tm_cq, g * BK, 0, full(s));
+    };
+    if (lane == 0)
+      for (int g = 0; g < pre; ++g) mbar_arrive_expect_tx(full(g), stage_tx(g));
+    __syncwarp();
+    if (lane < pre) issue_w(lane, 0);
+    else if (lane >= 8 && lane - 8 < pre) issue_w(lane - 8, 1);
+    griddep_wait();
+    if (lane < pre && lane < p.k_blocks) issue_cq(lane);
+    __syncwarp();
+    int g = pre;
     for (; g < total; ++g) {
       const int s = g % p.stages;
       const bool first = g < p.k_blocks;
       bool good = true;
       if (lane == 0) {
         if (g >= p.stages) good = mbar_wait(empty(s), ((g / p.stages) - 1) & 1, abort_flag);
-        if (good)
-          mbar_arrive_expect_tx(full(s), first ? ab::A_BYTES + ab::QR_BYTES + p.n_tile * BK * 2 : ab::A_BYTES);
+        if (good) mbar_arrive_expect_tx(full(s), stage_tx(g));
       }
       if (!__shfl_sync(0xffffffffu, good, 0)) break;
-      const uint32_t st = sbase + s * p.stage_bytes;
-      if (first) {
-        const int k0 = g * BK;
-        if (lane == 0) tma_load_2d(st, &tm_uq, k0, head * BM, full(s));
-        else if (lane == 1) tma_load_2d(st + ab::A_BYTES, &tm_qr, k0, head * p.d_r, full(s));
-        else if (lane == 2) tma_load_2d(st + 2 * ab::A_BYTES, &tm_cq, k0, 0, full(s));
-      } else {
-        // W_UK_h^T tile: latent columns [128 mt + 64 lane, +64) of k rows [64 kb, +64)
-        const int u = g - p.k_blocks, mt = u >> 1, kb = u & 1;
-        if (lane < 2) tma_load_2d(st + lane * (ab::A_BYTES / 2), &tm_uk, BM * mt + 64 * lane, head * BM + 64 * kb, full(s));
-      }
+      if (lane < 2) issue_w(g, lane);
+      else if (lane == 2 && first) issue_cq(g);
       __syncwarp();
     }
     if (lane == 0)  // drain: the MMA commits to the empty barriers have landed
@@ -353,6 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = 32 * sp + lane;  // accumulator row of this thread
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
     const int64_t q_row = static_cast<int64_t>(p.n_h) * (p.d_c + p.d_r);  // q elements per token
+    griddep_wait();  // positions are read and q written only once the previous kernel has finished
     mbar_wait_warp(p1_done, 0, abort_flag);
     tc_fence_after();
     // q_C,h row `row` -> B2 (MN-major, 128-byte swizzle): k = row, n = token
@@ -444,6 +488,8 @@ __device__ __forceinline__ float2 sum_splits2(const float *part, int splits, int
 // thread per element pair.
 __global__ void k_fin_append(const float *part, int splits, int T, int d_c, int d_r, double rope_base,
                              const int32_t *seq_idx, const int32_t *positions, CacheView cache) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
   const int t = blockIdx.y;
   const int D = d_c + d_r;
   const int e = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
@@ -464,6 +510,8 @@ __global__ void k_fin_append(const float *part, int splits, int T, int d_c, int 
 
 // dst[t][n] (bf16, row pitch ld) = sum of splits of part[.][t][n], n < N.
 __global__ void k_fin_store(const float *part, int splits, int T, int N, __nv_bfloat16 *dst, int64_t ld) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
   const int64_t stride = static_cast<int64_t>(T) * N;
   for (int64_t i = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); i < stride;
        i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {

@@ -36,6 +36,28 @@ std::atomic<uint64_t> g_launches{0};
 // Every kernel launch goes through this macro so the count is exact.
 #define MLA_LAUNCH(...) (g_launches.fetch_add(1, std::memory_order_relaxed), __VA_ARGS__)
 
+std::atomic<int> g_overlap{0};
+
+// Launch of a tensor-core kernel: plain, or with programmatic stream
+// serialization while launch overlap is on (the kernels wait for the grid
+// ahead of them with griddepcontrol.wait before touching its outputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_tc(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args &&...args) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_overlap.load(std::memory_order_relaxed) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 mla_status fail(mla_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 mla_status fail(mla_status s, const char *fmt, ...) {
   char buf[512];
@@ -51,6 +73,15 @@ mla_status cuda_check(const char *what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return MLA_OK;
+}
+
+// Status of a launch_tc() call: its own error, else any pending one.
+mla_status launched(cudaError_t e, const char *what) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+  return cuda_check(what);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -331,6 +362,7 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
   p.a_batch_rows = a_batch_rows;
   p.b_batch_cols = b_batch_cols;
   p.stages = G::stages_for(g.n_tile, g.m_tiles * g.n_tiles * g.batches * g.splits, sm_count());
+  p.prefetch = g_overlap.load(std::memory_order_relaxed);  // the kernel is correct either way
   const size_t smem = G::smem_for(g.n_tile, p.stages);
   static bool attr = false;
   if (!attr) {
@@ -339,8 +371,8 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
     attr = true;
   }
   dim3 grid(g.m_tiles, g.n_tiles, g.batches * g.splits);
-  MLA_LAUNCH(G::k_gemm<<<grid, G::NUM_THREADS, smem, st>>>(ta, ta2, tb, p));
-  return cuda_check("projection GEMM (tensor cores)");
+  return launched(launch_tc(G::k_gemm, grid, dim3(G::NUM_THREADS), smem, st, ta, ta2, tb, p),
+                  "projection GEMM (tensor cores)");
 }
 
 GemmShape append_shape(const mla_dims *d, int T) { return gemm_shape(d->d_c + d->d_r, T, d->d, 1, true); }
@@ -361,10 +393,9 @@ mla_status tc_append(const mla_dims *d, const void *h, const void *W_DKV, const 
   p.out = part;
   if ((s = launch_gemm(ta, ta2, tb, g, T, d->d_c, false, 0, 0, p, st)) != MLA_OK) return s;
   const int D = d->d_c + d->d_r;
-  MLA_LAUNCH(G::k_fin_append<<<dim3((D / 2 + 127) / 128, T), 128, 0, st>>>(part, g.splits, T, d->d_c, d->d_r,
-                                                                         d->rope_base, seq_idx, positions,
-                                                                         view_of(c)));
-  return cuda_check("append finalize");
+  return launched(launch_tc(G::k_fin_append, dim3((D / 2 + 127) / 128, T), dim3(128), 0, st, part, g.splits, T,
+                            d->d_c, d->d_r, d->rope_base, seq_idx, positions, view_of(c)),
+                  "append finalize");
 }
 
 struct AbsorbPlan {
@@ -403,8 +434,10 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   p.out = part;
   if ((s = launch_gemm(ta, ta, tb, a.cq, T, d->d_cq, false, 0, 0, p, st)) != MLA_OK) return s;
   const int64_t pairs = static_cast<int64_t>(T) * d->d_cq / 2;
-  MLA_LAUNCH(G::k_fin_store<<<static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256)), 256, 0, st>>>(
-      part, a.cq.splits, T, d->d_cq, cq, d->d_cq));
+  if ((s = launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
+                              dim3(256), 0, st, part, a.cq.splits, T, d->d_cq, cq, static_cast<int64_t>(d->d_cq)),
+                    "c_Q finalize")) != MLA_OK)
+    return s;
   if (a.uq.n_tile <= 128) {
     // one CTA per head: q_C,h = W_UQ_h c_Q, q_R,h = RoPE(W_QR_h c_Q), q_lat,h = W_UK_h^T q_C,h
     CUtensorMap tq, tr, tc, tk;
@@ -425,6 +458,7 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
     ap.q = static_cast<__nv_bfloat16 *>(q);
     ap.positions = positions;
     ap.rope_base = d->rope_base;
+    ap.prefetch = g_overlap.load(std::memory_order_relaxed);  // the kernel is correct either way
     const size_t smem = G::ab::smem(ap.n_tile, ap.stages);
     static bool attr = false;
     if (!attr) {
@@ -432,8 +466,8 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
         return cuda_check("absorb: set shared memory size");
       attr = true;
     }
-    MLA_LAUNCH(G::k_absorb_head<<<d->n_h, G::NUM_THREADS, smem, st>>>(tq, tr, tc, tk, ap));
-    return cuda_check("fused per-head absorb (tensor cores)");
+    return launched(launch_tc(G::k_absorb_head, dim3(d->n_h), dim3(G::NUM_THREADS), smem, st, tq, tr, tc, tk, ap),
+                    "fused per-head absorb (tensor cores)");
   }
   // [q_C ; q_R] = [W_UQ ; W_QR] c_Q: q_C to the workspace, q_R rotated into q
   if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
@@ -578,10 +612,12 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
       return cuda_check("decode: set shared memory size");
     attr_done = true;
   }
-  MLA_LAUNCH(D::k_decode<<<2 * nclusters, D::NUM_THREADS, D::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v[0], tm_v[1], p));
-  if ((s = cuda_check("decode (tensor cores)")) != MLA_OK) return s;
-  MLA_LAUNCH(D::k_combine<<<BJ * D::COMBINE_BLOCKS_PER_ROW, 128, 0, st>>>(p));
-  return cuda_check("decode combine");
+  if ((s = launched(launch_tc(D::k_decode, dim3(2 * nclusters), dim3(D::NUM_THREADS), D::SMEM_BYTES, st, tm_q,
+                              tm_k, tm_v[0], tm_v[1], p),
+                    "decode (tensor cores)")) != MLA_OK)
+    return s;
+  return launched(launch_tc(D::k_combine, dim3(BJ * D::COMBINE_BLOCKS_PER_ROW), dim3(128), 0, st, p),
+                  "decode combine");
 }
 
 }  // namespace
@@ -656,6 +692,13 @@ const char *mla_status_string(mla_status s) {
 const char *mla_last_error_message(void) { return g_msg.c_str(); }
 
 uint64_t mla_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+mla_status mla_set_launch_overlap(int32_t enable) {
+  g_overlap.store(enable != 0 ? 1 : 0, std::memory_order_relaxed);
+  return MLA_OK;
+}
+
+int32_t mla_get_launch_overlap(void) { return g_overlap.load(std::memory_order_relaxed); }
 
 int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   if (d == nullptr || !tc_geometry(d)) return 0;

@@ -26,6 +26,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ----------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel ahead of it on the stream is still running. griddep_wait() returns
+// once every grid it depends on has completed with its memory visible (at
+// once in a kernel launched without the attribute); nothing that kernel may
+// write, or that the kernels before it wrote, is touched before it.
+// griddep_launch_dependents() lets the next such kernel be scheduled as soon
+// as every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ cluster
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -56,7 +56,7 @@ _lib.mla_uses_tensor_cores.argtypes = [C.POINTER(Dims), C.c_int32]
 _lib.mla_uses_tensor_cores.restype = C.c_int32
 _lib.mla_kernel_launches.restype = C.c_uint64
 for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj",
-           "mla_get_device_error"):
+           "mla_get_device_error", "mla_set_launch_overlap", "mla_get_launch_overlap"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -170,6 +170,18 @@ def mla_get_device_error(stream=None) -> int:
 
 def status_string(s: int) -> str:
     return _lib.mla_status_string(s).decode()
+
+
+def set_launch_overlap(enable: bool) -> None:
+    """Process-wide: launch the tensor-core kernels with programmatic stream
+    serialization, so that each may set up and start streaming its weights
+    while the kernel ahead of it finishes (results are identical). The weights
+    of a call must not be written by the work enqueued just before it."""
+    _check(_lib.mla_set_launch_overlap(1 if enable else 0), "mla_set_launch_overlap")
+
+
+def get_launch_overlap() -> bool:
+    return bool(_lib.mla_get_launch_overlap())
 
 
 def kernel_launches() -> int:

@@ -28,3 +28,13 @@ def test_library_exports_every_declared_symbol():
     lib.mla_status_string.restype = ctypes.c_char_p
     assert lib.mla_status_string(0) == b"MLA_OK"
     assert lib.mla_status_string(6) == b"MLA_ERR_DEVICE_DATA"
+
+
+def test_launch_overlap_switch_round_trips():
+    from mla_latent_kv_33_b200 import build
+    lib = ctypes.CDLL(build.build())
+    assert lib.mla_get_launch_overlap() == 0  # off by default
+    assert lib.mla_set_launch_overlap(1) == 0
+    assert lib.mla_get_launch_overlap() == 1
+    assert lib.mla_set_launch_overlap(0) == 0
+    assert lib.mla_get_launch_overlap() == 0
