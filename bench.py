@@ -171,6 +171,16 @@ def upload(x, torch, dev):
     return W, cache_t, bt
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over the process group (every
+    rank gets the result): the job is as slow as its slowest replica."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from mla_latent_kv_33_b200 import mla
@@ -340,10 +350,7 @@ def run_ours(args, rank, world, local_rank):
 
     step_ms = ms_total / args.steps
     if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([step_ms, dec_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        step_ms, dec_ms, e2e_ms = (float(v) for v in tt.tolist())
+        step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], dev)
     del graph_1, graph_k
     return {"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
             "launch_mode": ("eager" if args.eager else "cuda_graph") + ("" if args.no_overlap else "+overlap"),
