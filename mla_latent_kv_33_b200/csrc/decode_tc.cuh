@@ -684,6 +684,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       const float inv = 1.f / ltot;
       const float lse_v = m_ref * p.scale + logf(ltot);
       const int head = HPC * rank + row;
+      // A TMEM load gives each thread 32 columns of its own head, so a warp
+      // holds 32 heads x 32 columns. It transposes them, 16 columns at a time,
+      // through its threads' own 2 KB of the exchange buffer (free here: every
+      // thread has passed the last P exchange), so that a store instruction
+      // writes 8 heads x 16 contiguous columns rather than 32 heads x 4 or 8.
+      // The 16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3) of the
+      // row's 64 bytes: both the row writes and the column reads are free of
+      // bank conflicts.
+      float *stg = reinterpret_cast<float *>(smem + OFF_XBUF + 2048 * sp);
+      const int head_w = HPC * rank + 32 * (sp & 1);  // head of the warp's row 0
+      const int sw_w = (lane >> 1) & 3;
+      const int r0 = lane >> 2, c4 = lane & 3;
 #pragma unroll 1
       for (int q4 = 0; q4 < 8; ++q4) {
         const int j = q4 >> 2, part = q4 & 3;
@@ -691,22 +703,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         tmem_ld32(lane_addr + 128 * j + 32 * part, o);
         tmem_wait_ld();
         const int col = 256 * j + 128 * half + 32 * part;
-        if (pc.single) {
-          uint4 *dst = reinterpret_cast<uint4 *>(p.o_lat + (static_cast<int64_t>(pc.bj) * HEADS + head) * DC + col);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
+        for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(o[8 * v + 2 * e]) * inv, __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
-            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4 *>(stg + 16 * lane + 4 * (k ^ sw_w)) =
+                make_float4(__uint_as_float(o[16 * h2 + 4 * k]) * inv, __uint_as_float(o[16 * h2 + 4 * k + 1]) * inv,
+                            __uint_as_float(o[16 * h2 + 4 * k + 2]) * inv, __uint_as_float(o[16 * h2 + 4 * k + 3]) * inv);
+          __syncwarp();
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const int r = r0 + 8 * k2;
+            const float4 v = *reinterpret_cast<const float4 *>(stg + 16 * r + 4 * (c4 ^ ((r >> 1) & 3)));
+            const int64_t at = (static_cast<int64_t>(pc.single ? pc.bj : pc.slot) * HEADS + head_w + r) * DC + col +
+                               16 * h2 + 4 * c4;
+            if (pc.single)
+              *reinterpret_cast<uint2 *>(p.o_lat + at) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+            else
+              *reinterpret_cast<float4 *>(p.part_o + at) = v;
           }
-        } else {
-          float4 *dst = reinterpret_cast<float4 *>(p.part_o + (static_cast<int64_t>(pc.slot) * HEADS + head) * DC + col);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                 __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+          __syncwarp();  // the rows are rewritten by the next half
         }
       }
       if (half == 0) {
