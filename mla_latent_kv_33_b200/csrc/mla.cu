@@ -84,6 +84,22 @@ mla_status launched(cudaError_t e, const char *what) {
   return cuda_check(what);
 }
 
+// cudaFuncSetAttribute applies to the current device: a kernel's dynamic
+// shared memory limit is raised once per device (bit `device` of its mask).
+enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_KERNELS = 3 };
+std::atomic<uint64_t> g_smem_raised[SMEM_KERNELS];
+
+mla_status raise_smem_limit(const void *kernel, SmemKernel which, int bytes, const char *what) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_check(what);
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit != 0 && (g_smem_raised[which].load(std::memory_order_acquire) & bit) != 0) return MLA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return cuda_check(what);
+  g_smem_raised[which].fetch_or(bit, std::memory_order_release);
+  return MLA_OK;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t elem_size(const mla_dims *d) { return d->dtype == MLA_BF16 ? 2 : 4; }
@@ -364,12 +380,9 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
   p.stages = G::stages_for(g.n_tile, g.m_tiles * g.n_tiles * g.batches * g.splits, sm_count());
   p.prefetch = g_overlap.load(std::memory_order_relaxed);  // the kernel is correct either way
   const size_t smem = G::smem_for(g.n_tile, p.stages);
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(G::k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
-      return cuda_check("gemm: set shared memory size");
-    attr = true;
-  }
+  mla_status s = raise_smem_limit(reinterpret_cast<const void *>(G::k_gemm), SMEM_GEMM, 232448,
+                                  "gemm: set shared memory size");
+  if (s != MLA_OK) return s;
   dim3 grid(g.m_tiles, g.n_tiles, g.batches * g.splits);
   return launched(launch_tc(G::k_gemm, grid, dim3(G::NUM_THREADS), smem, st, ta, ta2, tb, p),
                   "projection GEMM (tensor cores)");
@@ -460,12 +473,9 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
     ap.rope_base = d->rope_base;
     ap.prefetch = g_overlap.load(std::memory_order_relaxed);  // the kernel is correct either way
     const size_t smem = G::ab::smem(ap.n_tile, ap.stages);
-    static bool attr = false;
-    if (!attr) {
-      if (cudaFuncSetAttribute(G::k_absorb_head, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
-        return cuda_check("absorb: set shared memory size");
-      attr = true;
-    }
+    if ((s = raise_smem_limit(reinterpret_cast<const void *>(G::k_absorb_head), SMEM_ABSORB, 232448,
+                              "absorb: set shared memory size")) != MLA_OK)
+      return s;
     return launched(launch_tc(G::k_absorb_head, dim3(d->n_h), dim3(G::NUM_THREADS), smem, st, tq, tr, tc, tk, ap),
                     "fused per-head absorb (tensor cores)");
   }
@@ -606,12 +616,9 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan_bytes);
   p.part_lse = p.part_o + slots * D::HEADS * D::DC;
 
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(D::k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES) != cudaSuccess)
-      return cuda_check("decode: set shared memory size");
-    attr_done = true;
-  }
+  if ((s = raise_smem_limit(reinterpret_cast<const void *>(D::k_decode), SMEM_DECODE, D::SMEM_BYTES,
+                            "decode: set shared memory size")) != MLA_OK)
+    return s;
   if ((s = launched(launch_tc(D::k_decode, dim3(2 * nclusters), dim3(D::NUM_THREADS), D::SMEM_BYTES, st, tm_q,
                               tm_k, tm_v[0], tm_v[1], p),
                     "decode (tensor cores)")) != MLA_OK)
