@@ -34,29 +34,32 @@ class OrcCache(C.Structure):
 _P = C.c_void_p
 
 
+def bind(L):
+    """Declare the C signatures on a loaded liboracle (argument marshalling)."""
+    L.orc_rope.argtypes = [_P, C.c_int, C.c_double, C.c_double]
+    L.orc_slot.argtypes = [C.POINTER(OrcCache), C.c_int32, C.c_int64]
+    L.orc_slot.restype = C.c_int64
+    L.orc_append.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, C.c_int, _P]
+    L.orc_absorb_q.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, _P, _P, C.c_int, _P, _P]
+    L.orc_decode.argtypes = [C.POINTER(OrcDims), _P, C.POINTER(OrcCache), _P, C.c_int, C.c_int,
+                             _P, _P, _P, C.c_int]
+    L.orc_decode.restype = C.c_int
+    L.orc_attend_range.argtypes = [C.POINTER(OrcDims), _P, C.POINTER(OrcCache), C.c_int32,
+                                   C.c_int64, C.c_int64, _P, _P]
+    L.orc_combine.argtypes = [C.c_int, C.c_int, _P, _P, _P, _P]
+    L.orc_out_proj.argtypes = [C.POINTER(OrcDims), _P, _P, C.c_int, _P]
+    L.orc_decode_order_a.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, C.POINTER(OrcCache),
+                                     _P, C.c_int, C.c_int, _P, _P, C.c_int]
+    L.orc_decode_order_a.restype = C.c_int
+    L.orc_set_threads.argtypes = [C.c_int]
+    L.orc_max_threads.restype = C.c_int
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = C.CDLL(path)
-        L.orc_rope.argtypes = [_P, C.c_int, C.c_double, C.c_double]
-        L.orc_slot.argtypes = [C.POINTER(OrcCache), C.c_int32, C.c_int64]
-        L.orc_slot.restype = C.c_int64
-        L.orc_append.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, C.c_int, _P]
-        L.orc_absorb_q.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, _P, _P, C.c_int, _P, _P]
-        L.orc_decode.argtypes = [C.POINTER(OrcDims), _P, C.POINTER(OrcCache), _P, C.c_int, C.c_int,
-                                 _P, _P, _P, C.c_int]
-        L.orc_decode.restype = C.c_int
-        L.orc_attend_range.argtypes = [C.POINTER(OrcDims), _P, C.POINTER(OrcCache), C.c_int32,
-                                       C.c_int64, C.c_int64, _P, _P]
-        L.orc_combine.argtypes = [C.c_int, C.c_int, _P, _P, _P, _P]
-        L.orc_out_proj.argtypes = [C.POINTER(OrcDims), _P, _P, C.c_int, _P]
-        L.orc_decode_order_a.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, C.POINTER(OrcCache),
-                                         _P, C.c_int, C.c_int, _P, _P, C.c_int]
-        L.orc_decode_order_a.restype = C.c_int
-        L.orc_set_threads.argtypes = [C.c_int]
-        L.orc_max_threads.restype = C.c_int
-        _lib = L
+        _lib = bind(C.CDLL(_build.build()))
     return _lib
 
 
