@@ -115,8 +115,9 @@ mla_status mla_cache_append(const mla_dims *dims, const void *h, const void *W_D
  *   h [T][d]  W_DQ [d_cq][d]  W_UQ [n_h*d_h][d_cq]  W_QR [n_h*d_r][d_cq]
  *   W_UK [n_h*d_h][d_c]  positions [T] int32 device
  *   q (output) [T][n_h][D] = [q_lat | q_R] per head, storage dtype.
- * c_Q and q_C are tensor-core operands and are rounded to the storage dtype
- * in the workspace; q is rounded once. */
+ * c_Q and q_C are tensor-core operands and are rounded once to the storage
+ * dtype: c_Q in the workspace, q_C in shared memory (at most 128 token rows,
+ * one CTA per head) or in the workspace (more rows); q is rounded once. */
 mla_status mla_absorb_q(const mla_dims *dims, const void *h, const void *W_DQ, const void *W_UQ,
                         const void *W_QR, const void *W_UK, const int32_t *positions, int32_t T,
                         void *q, void *ws, size_t ws_bytes, void *stream);
@@ -202,7 +203,9 @@ mla_status mla_set_launch_overlap(int32_t enable);
 int32_t mla_get_launch_overlap(void);
 
 /* Number of kernels this library has launched in this process (all devices,
- * all threads). Lets callers count launches inside a timed region. */
+ * all threads), counted when they are enqueued; a launch captured into a CUDA
+ * graph counts once at capture, however often the graph is replayed. Lets
+ * callers count launches inside a timed region. */
 uint64_t mla_kernel_launches(void);
 
 #ifdef __cplusplus
