@@ -1,0 +1,72 @@
+"""Host-side pieces of bench.py, on CPU: the clock summary keeps only the
+samples of the timed region and reports every throttle reason it saw; the
+DRAM traffic figure is taken from the committed profile only while the
+profiled source is unchanged; the reported config names the workload."""
+import hashlib
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from mla_latent_kv_33_b200 import synth  # noqa: E402
+
+
+def _line(sm, smax=1965, reasons=("Not Active",) * 4):
+    return f"0, {sm}, {smax}, 700.00, 0x0, " + ", ".join(reasons) + "\n"
+
+
+def test_clock_summary_keeps_the_timed_window():
+    c = bench.ClockSampler("0")
+    c.samples = [(0.0, _line(1200)), (1.0, _line(1965)), (1.1, _line(1950)), (1.2, _line(1965)), (3.0, _line(900))]
+    c.mark(0.95, 1.25)
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["samples"] == 3 and s["reasons"] == []
+
+
+def test_clock_summary_reports_throttle_reasons():
+    c = bench.ClockSampler("0")
+    c.samples = [(1.0, _line(1400, reasons=("Not Active", "Not Active", "Not Active", "Active"))),
+                 (1.1, _line(1300, reasons=("Active", "Not Active", "Not Active", "Not Active")))]
+    c.mark(0.9, 1.2)
+    assert c.summary()["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_summary_short_region_takes_the_nearest_sample():
+    c = bench.ClockSampler("0")
+    c.samples = [(0.0, _line(1000)), (1.0, _line(1800)), (2.0, _line(1100))]
+    c.mark(1.001, 1.002)  # shorter than the sampling period
+    s = c.summary()
+    assert s["samples"] == 1 and s["sm_mhz"] == 1800.0
+
+
+def test_clock_summary_without_samples():
+    c = bench.ClockSampler("0")
+    c.samples = [(1.0, "garbage\n")]
+    assert c.summary() is None
+
+
+def test_decode_traffic_follows_the_profiled_source(tmp_path, monkeypatch):
+    got = bench.decode_traffic("v2_b64_paged")
+    doc = open(os.path.join(ROOT, "profiles", "k_decode_v2_b64_paged.md")).read()
+    src = open(os.path.join(ROOT, "mla_latent_kv_33_b200", "csrc", "decode_tc.cuh"), "rb").read()
+    fields = dict(l.split(": ", 1) for l in doc.splitlines() if ": " in l and l.split(": ", 1)[0] in
+                  ("traffic_bytes_per_launch", "decode_source_sha256_16"))
+    if fields["decode_source_sha256_16"].strip() == hashlib.sha256(src).hexdigest()[:16]:
+        assert got == int(fields["traffic_bytes_per_launch"])
+    else:
+        assert got is None
+    assert bench.decode_traffic("no_such_workload") is None
+
+
+def test_config_names_the_workload():
+    w = synth.shrink(synth.WORKLOADS["v2_b64_paged"], B=3, L_lo=5, L_hi=130, d=64, d_cq=32)
+    x = synth.generate(w)
+    cfg = bench.config_of(w, 1, x)
+    assert cfg["workload"] == "v2_b64_paged" and cfg["batch"] == 3 and cfg["paged"] is True
+    assert cfg["seq_len_min"] == int(np.min(x.seq_lens)) and cfg["parallelism"] == "replicas1"
+    assert "model" not in cfg
