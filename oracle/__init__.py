@@ -51,6 +51,8 @@ def bind(L):
     L.orc_decode_order_a.argtypes = [C.POINTER(OrcDims), _P, _P, _P, _P, C.POINTER(OrcCache),
                                      _P, C.c_int, C.c_int, _P, _P, C.c_int]
     L.orc_decode_order_a.restype = C.c_int
+    L.orc_o_proj.argtypes = [_P, C.c_int, C.c_int, _P, C.c_int, _P]
+    L.orc_absorb_wo.argtypes = [C.POINTER(OrcDims), _P, _P, _P]
     L.orc_set_threads.argtypes = [C.c_int]
     L.orc_max_threads.restype = C.c_int
     return L
@@ -188,6 +190,24 @@ def out_proj(p: OrcDims, o_lat, W_UV):
     o = np.zeros((T, p.n_h * p.d_h), np.float64)
     lib().orc_out_proj(C.byref(p), _ptr(o_lat), _ptr(W_UV), T, _ptr(o))
     return o
+
+
+def o_proj(W, x):
+    """y[t] = W x[t] (walk-through step 5 with W = W_O and x = the concatenated
+    head outputs; or W = W_OV from absorb_wo and x = o_lat flattened)."""
+    W = _f64(W)
+    x = _f64(x).reshape(-1, W.shape[1])
+    y = np.empty((x.shape[0], W.shape[0]))
+    lib().orc_o_proj(_ptr(W), W.shape[0], W.shape[1], _ptr(x), x.shape[0], _ptr(y))
+    return y
+
+
+def absorb_wo(p: OrcDims, W_O, W_UV):
+    """W_OV (d x n_h*d_c): W_UV absorbed into W_O."""
+    W_O, W_UV = _f64(W_O), _f64(W_UV)
+    W_OV = np.empty((p.d, p.n_h * p.d_c))
+    lib().orc_absorb_wo(C.byref(p), _ptr(W_O), _ptr(W_UV), _ptr(W_OV))
+    return W_OV
 
 
 def decode_order_a(p: OrcDims, q_C, q_R, W_UK, W_UV, cache: Cache, seq_lens, n_q, pairs=None):

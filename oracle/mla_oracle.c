@@ -280,6 +280,31 @@ void orc_out_proj(const orc_dims *p, const double *o_lat, const double *W_UV, in
                  o + (int64_t)t * p->n_h * p->d_h + (int64_t)hh * p->d_h);
 }
 
+/* Step 5 of the walk-through (section 1, "整合"): the n_h head outputs of a
+ * token, concatenated (n_h * d_h numbers), are projected back to the model
+ * width by W_O (d x n_h*d_h): y_t = W x_t for every token row t. The same
+ * routine applies the absorbed matrix of orc_absorb_wo to o_lat. */
+void orc_o_proj(const double *W, int rows, int cols, const double *x, int T, double *y) {
+  for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)t * cols, y + (int64_t)t * rows);
+}
+
+/* W_UV absorbed into the output projection (DeepSeek-V2 explainer, section 3
+ * remark; MLA walk-through, section 3 order B): since o_h = W_UV_h o_lat,h,
+ * W_O [o_1; ...; o_n_h] = W_OV [o_lat,1; ...; o_lat,n_h] with
+ *   W_OV[r][h*d_c + j] = sum_i W_O[r][h*d_h + i] W_UV[h*d_h + i][j],
+ * a d x n_h*d_c matrix. W_O is d x n_h*d_h, W_UV is n_h*d_h x d_c. */
+void orc_absorb_wo(const orc_dims *p, const double *W_O, const double *W_UV, double *W_OV) {
+  const int64_t ko = (int64_t)p->n_h * p->d_h, kv = (int64_t)p->n_h * p->d_c;
+  for (int r = 0; r < p->d; ++r)
+    for (int hh = 0; hh < p->n_h; ++hh)
+      for (int j = 0; j < p->d_c; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < p->d_h; ++i)
+          acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[((int64_t)hh * p->d_h + i) * p->d_c + j];
+        W_OV[r * kv + (int64_t)hh * p->d_c + j] = acc;
+      }
+}
+
 /* Order A (training form, section 3): decompress per head
  *   k_C,i = W_UK_h c_KV_i, v_i = W_UV_h c_KV_i,
  * score = scale * ([q_C ; q_R] . [k_C,i ; k_R,i]) in d_h + d_r dims,

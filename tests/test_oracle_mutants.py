@@ -39,6 +39,12 @@ MUTANTS = [
     ("bf16 bits shifted", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
     ("paged slot ignores the block offset", "return blk * c->block_size + pos % c->block_size;",
      "return blk * c->block_size;"),
+    ("W_O absorption reads W_UV transposed",
+     "acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[((int64_t)hh * p->d_h + i) * p->d_c + j];",
+     "acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[(int64_t)hh * p->d_h * p->d_c + (int64_t)j * p->d_h + i];"),
+    ("output projection skips a token row",
+     "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)t * cols, y + (int64_t)t * rows);",
+     "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)(t > 0 ? t - 1 : 0) * cols, y + (int64_t)t * rows);"),
 ]
 
 

@@ -279,6 +279,33 @@ def test_out_proj_matches_library(orc):
     assert np.allclose(o, ref, rtol=1e-13, atol=1e-14)
 
 
+# ------------------------------------ output projection W_O (next row) ----
+
+def test_o_proj_matches_library(orc):
+    # walk-through step 5: the concatenated head outputs times W_O (d x n_h d_h)
+    rng = np.random.default_rng(12)
+    W_O = rng.standard_normal((7, 12))
+    o = rng.standard_normal((5, 12))
+    assert np.allclose(orc.o_proj(W_O, o), o @ W_O.T, rtol=1e-13, atol=1e-14)
+
+
+def test_absorbed_w_o_matches_library_and_the_two_stage_readout(orc):
+    # W_UV absorbed into W_O: W_OV[r][h d_c + j] = sum_i W_O[r][h d_h + i] W_UV[h d_h + i][j]
+    rng = np.random.default_rng(13)
+    n_h, d_h, d_c, d = 3, 4, 6, 7
+    p = orc.dims(d=d, n_h=n_h, d_h=d_h, d_c=d_c, d_cq=8, d_r=2)
+    W_O = rng.standard_normal((d, n_h * d_h))
+    W_UV = rng.standard_normal((n_h * d_h, d_c))
+    W_OV = orc.absorb_wo(p, W_O, W_UV)
+    ref = np.einsum("rhi,hij->rhj", W_O.reshape(d, n_h, d_h), W_UV.reshape(n_h, d_h, d_c)).reshape(d, n_h * d_c)
+    assert np.allclose(W_OV, ref, rtol=1e-13, atol=1e-14)
+    # reading out in latent space with W_OV equals decompressing with W_UV, then W_O
+    o_lat = rng.standard_normal((5, n_h, d_c))
+    one_stage = orc.o_proj(W_OV, o_lat.reshape(5, n_h * d_c))
+    two_stage = orc.o_proj(W_O, orc.out_proj(p, o_lat, W_UV))
+    assert np.allclose(one_stage, two_stage, rtol=1e-12, atol=1e-13)
+
+
 def test_bf16_cache_read_is_exact(orc):
     # the oracle reads bf16 storage as the exact real value of those bits
     vals = np.array([1.0, -2.5, 3.140625, 1e-3, 65280.0], np.float32)
