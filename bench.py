@@ -171,6 +171,11 @@ def upload(x, torch, dev):
     return W, cache_t, bt
 
 
+def percentiles_us(ms_list):
+    """p10, p50 and p90 of per-step durations given in ms, in µs (this rank)."""
+    return [float(v) * 1e3 for v in np.percentile(np.asarray(ms_list, dtype=np.float64), [10, 50, 90])]
+
+
 def max_over_ranks(values, device):
     """Element-wise max of per-rank timings over the process group (every
     rank gets the result): the job is as slow as its slowest replica."""
@@ -298,7 +303,9 @@ def run_ours(args, rank, world, local_rank):
     launches = mla.kernel_launches() - launches0 + launches_k
     barrier()
     ms_total = t0.elapsed_time(t1)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    dec_list = [a.elapsed_time(b) for a, b in ev_dec]
+    dec_ms = float(np.mean(dec_list))
+    dec_pct = percentiles_us(dec_list)
 
     # End to end through the public API: every step copies its inputs in from
     # pinned host memory and its output o back, inside the timed region. The
@@ -352,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], dev)
     del graph_1, graph_k
-    return {"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+    return {"step_ms": step_ms, "dec_ms": dec_ms, "dec_pct": dec_pct, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
             "launch_mode": ("eager" if args.eager else "cuda_graph") + ("" if args.no_overlap else "+overlap"),
             "launches": launches, "clocks": clk.summary(), "x": x, "w": w,
             "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
@@ -486,7 +493,8 @@ def main():
         "metric": METRIC, "value": us, "unit": "µs/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world, x),
-        "decode_us": r["dec_ms"] * 1e3, "cache_gbs": cache_gbs, "tflops": tflops,
+        "decode_us": r["dec_ms"] * 1e3, "decode_us_p10_p50_p90": r["dec_pct"], "cache_gbs": cache_gbs,
+        "tflops": tflops,
         "tokens_per_s": world * w.T / (r["step_ms"] * 1e-3),
         "roofline": roof,
         "e2e": {"value": r["e2e_ms"] * 1e3, "unit": "µs/step", "h2d_bytes_per_step": r["h2d"],

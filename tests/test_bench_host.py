@@ -70,3 +70,9 @@ def test_config_names_the_workload():
     assert cfg["workload"] == "v2_b64_paged" and cfg["batch"] == 3 and cfg["paged"] is True
     assert cfg["seq_len_min"] == int(np.min(x.seq_lens)) and cfg["parallelism"] == "replicas1"
     assert "model" not in cfg
+
+
+def test_percentiles_of_step_durations():
+    ms = [0.1 * k for k in range(1, 101)]  # 0.1 .. 10 ms
+    p10, p50, p90 = bench.percentiles_us(ms)
+    assert abs(p10 - 1090.0) < 1e-6 and abs(p50 - 5050.0) < 1e-6 and abs(p90 - 9010.0) < 1e-6
