@@ -168,10 +168,18 @@ mla_status mla_decode_noalloc(const mla_dims *dims, const void *q, const mla_cac
 mla_status mla_out_proj(const mla_dims *dims, const void *o_lat, const void *W_UV, int32_t T,
                         void *o, void *ws, size_t ws_bytes, void *stream);
 
+/* Output projection (MLA walk-through, section 1 step 5: the n_h head outputs
+ * of a token, concatenated, are projected back to the model width):
+ *   y[t][r] = sum_k W_O[r][k] o[t][k],  k < n_h*d_h.
+ *   o [T][n_h*d_h] (the output of mla_out_proj)   W_O [d][n_h*d_h]
+ *   y (output) [T][d], storage dtype, rounded once from fp32 sums. */
+mla_status mla_o_proj(const mla_dims *dims, const void *o, const void *W_O, int32_t T, void *y, void *ws,
+                      size_t ws_bytes, void *stream);
+
 /* Scratch size in bytes for one call of `op` (MLA_OP_*). `rows` is T for
  * append/absorb/out_proj and B for decode; n_q and max_seq_len are used by
  * decode only (max_seq_len may be 0 for the tensor-core path). */
-enum { MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3 };
+enum { MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3, MLA_OP_O_PROJ = 4 };
 size_t mla_workspace_size(const mla_dims *dims, int32_t op, int32_t rows, int32_t n_q,
                           int64_t max_seq_len);
 

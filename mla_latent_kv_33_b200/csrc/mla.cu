@@ -255,6 +255,21 @@ mla_status simt_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV,
   return cuda_check("out_proj (CUDA cores)");
 }
 
+template <typename T>
+mla_status simt_o_proj(const mla_dims *d, const void *o, const void *W_O, int Tn, void *y, void *ws, cudaStream_t st) {
+  // y[t][r] = sum_k W_O[r][k] o[t][k]
+  const int64_t HD = static_cast<int64_t>(d->n_h) * d->d_h;
+  float *acc = static_cast<float *>(ws);  // [T][d]
+  launch_linear<T>(static_cast<const T *>(W_O), 0, HD, 1, o, false, 0, HD, acc, 0, d->d, d->d, static_cast<int>(HD),
+                   Tn, 1, st);
+  const int64_t n = static_cast<int64_t>(Tn) * d->d;
+  const int64_t blocks = (n + 255) / 256;
+  MLA_LAUNCH(mla::k_simt_store<T><<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(acc, static_cast<T *>(y), n));
+  return cuda_check("o_proj (CUDA cores)");
+}
+
+size_t simt_o_proj_ws(const mla_dims *d, int Tn) { return sizeof(float) * static_cast<size_t>(Tn) * d->d; }
+
 size_t simt_out_proj_ws(const mla_dims *d, int Tn) {
   return sizeof(float) * static_cast<size_t>(Tn) * d->n_h * d->d_h;
 }
@@ -526,6 +541,31 @@ mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, i
   return launch_gemm(ta, ta, tb, g, T, d->d_h, false, d->d_h, d->d_c, p, st);
 }
 
+// y = W_O o: split-K over the n_h*d_h columns, fp32 partials, then summed to
+// bf16 (the c_Q = W_DQ h pattern with W_O in place of W_DQ).
+GemmShape o_proj_shape(const mla_dims *d, int T) { return gemm_shape(d->d, T, d->n_h * d->d_h, 1, true); }
+
+size_t tc_o_proj_ws(const mla_dims *d, int T) { return gemm_part_bytes(o_proj_shape(d, T), T); }
+
+mla_status tc_o_proj(const mla_dims *d, const void *o, const void *W_O, int T, void *y, void *ws, cudaStream_t st) {
+  const GemmShape g = o_proj_shape(d, T);
+  const int HD = d->n_h * d->d_h;
+  float *part = static_cast<float *>(ws);
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_O, HD, d->d, HD * 2ull, 64, 128, "W_O")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, o, HD, T, HD * 2ull, 64, g.n_tile, "o")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = part;
+  if ((s = launch_gemm(ta, ta, tb, g, T, d->d, false, 0, 0, p, st)) != MLA_OK) return s;
+  const int64_t pairs = static_cast<int64_t>(T) * d->d / 2;
+  return launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
+                            dim3(256), 0, st, part, g.splits, T, d->d, static_cast<__nv_bfloat16 *>(y),
+                            static_cast<int64_t>(d->d)),
+                  "o_proj finalize");
+}
+
 // ------------------------------------------------- tensor-core decode ----
 
 // Clusters of two CTAs that can be resident at once (a pair must share a GPC,
@@ -709,7 +749,7 @@ int32_t mla_get_launch_overlap(void) { return g_overlap.load(std::memory_order_r
 
 int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   if (d == nullptr || !tc_geometry(d)) return 0;
-  return (op >= MLA_OP_APPEND && op <= MLA_OP_OUT_PROJ) ? 1 : 0;
+  return (op >= MLA_OP_APPEND && op <= MLA_OP_O_PROJ) ? 1 : 0;
 }
 
 size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len) {
@@ -721,6 +761,7 @@ size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n
     case MLA_OP_ABSORB: return tc ? tc_absorb_ws(d, rows) : simt_absorb_ws(d, rows);
     case MLA_OP_DECODE: return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count()) : 0;
     case MLA_OP_OUT_PROJ: return tc ? tc_out_proj_ws(d, rows) : simt_out_proj_ws(d, rows);
+    case MLA_OP_O_PROJ: return tc ? tc_o_proj_ws(d, rows) : simt_o_proj_ws(d, rows);
   }
   return 0;
 }
@@ -832,6 +873,23 @@ mla_status mla_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, 
   if (tc_geometry(d)) return tc_out_proj(d, o_lat, W_UV, T, o, ws, st);
   if (d->dtype == MLA_BF16) return simt_out_proj<__nv_bfloat16>(d, o_lat, W_UV, T, o, ws, st);
   return simt_out_proj<float>(d, o_lat, W_UV, T, o, ws, st);
+}
+
+mla_status mla_o_proj(const mla_dims *d, const void *o, const void *W_O, int32_t T, void *y, void *ws,
+                      size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!o || !W_O || !y) return fail(MLA_ERR_INVALID_ARG, "o_proj: NULL tensor argument");
+  if (!aligned16(o) || !aligned16(W_O) || !aligned16(y))
+    return fail(MLA_ERR_INVALID_ARG, "o_proj: tensors must be 16-byte aligned");
+  if (d->d % 2 != 0) return fail(MLA_ERR_UNSUPPORTED, "o_proj: d must be even");
+  const size_t need = mla_workspace_size(d, MLA_OP_O_PROJ, T, 1, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "o_proj needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_o_proj(d, o, W_O, T, y, ws, st);
+  if (d->dtype == MLA_BF16) return simt_o_proj<__nv_bfloat16>(d, o, W_O, T, y, ws, st);
+  return simt_o_proj<float>(d, o, W_O, T, y, ws, st);
 }
 
 }  // extern "C"

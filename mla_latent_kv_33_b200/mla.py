@@ -23,7 +23,7 @@ _lib = C.CDLL(LIB_PATH)
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA, MLA_ERR_TIMEOUT, \
     MLA_ERR_DEVICE_DATA = range(7)
 MLA_BF16, MLA_FP32 = 0, 1
-OP_APPEND, OP_ABSORB, OP_DECODE, OP_OUT_PROJ = range(4)
+OP_APPEND, OP_ABSORB, OP_DECODE, OP_OUT_PROJ, OP_O_PROJ = range(5)
 
 
 class Dims(C.Structure):
@@ -45,6 +45,7 @@ _lib.mla_absorb_q.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, C.c_int32
 _lib.mla_decode.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P,
                             C.c_int32, _P, _S, _P]
 _lib.mla_out_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
+_lib.mla_o_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
 _lib.mla_decode_noalloc.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P, _P]
 _lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64]
 _lib.mla_workspace_size.restype = C.c_size_t
@@ -55,7 +56,7 @@ _lib.mla_last_error_message.restype = C.c_char_p
 _lib.mla_uses_tensor_cores.argtypes = [C.POINTER(Dims), C.c_int32]
 _lib.mla_uses_tensor_cores.restype = C.c_int32
 _lib.mla_kernel_launches.restype = C.c_uint64
-for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj",
+for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj", "mla_o_proj",
            "mla_get_device_error", "mla_set_launch_overlap", "mla_get_launch_overlap"):
     getattr(_lib, _f).restype = C.c_int
 
@@ -161,6 +162,13 @@ def mla_out_proj(p: Dims, o_lat, W_UV, o, ws=None, stream=None):
     ws, nbytes = _ws(p, OP_OUT_PROJ, T, 1, ws)
     _check(_lib.mla_out_proj(C.byref(p), _ptr(o_lat), _ptr(W_UV), T, _ptr(o), _ptr(ws), nbytes,
                              _stream(stream)), "mla_out_proj")
+
+
+def mla_o_proj(p: Dims, o, W_O, y, ws=None, stream=None):
+    T = o.shape[0]
+    ws, nbytes = _ws(p, OP_O_PROJ, T, 1, ws)
+    _check(_lib.mla_o_proj(C.byref(p), _ptr(o), _ptr(W_O), T, _ptr(y), _ptr(ws), nbytes, _stream(stream)),
+           "mla_o_proj")
 
 
 def mla_get_device_error(stream=None) -> int:

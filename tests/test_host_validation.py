@@ -110,6 +110,17 @@ def test_absorb_and_out_proj_arguments(m):
     assert op(C.byref(v2(m, dtype="fp32")), A, A, 64, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
 
 
+def test_o_proj_arguments(m):
+    d = v2(m)
+    op = m._lib.mla_o_proj
+    assert op(C.byref(d), A, A, 0, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
+    assert op(C.byref(d), A, None, 64, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
+    assert op(C.byref(d), A, A, 64, MIS, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG and "aligned" in last_msg(m)
+    need = m._lib.mla_workspace_size(C.byref(d), m.OP_O_PROJ, 64, 1, 0)
+    assert 0 < need < 1 << 30  # split-K fp32 partials of the 5120 x 64 output
+    assert op(C.byref(d), A, A, 64, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
+
+
 def test_decode_arguments(m):
     d = v2(m)
     assert decode(m, d, B=0) == m.MLA_ERR_INVALID_ARG
@@ -147,7 +158,7 @@ def test_workspace_sizes(m):
 
 def test_tensor_core_geometry_switch(m):
     d = v2(m)
-    assert all(m._lib.mla_uses_tensor_cores(C.byref(d), op) == 1 for op in range(4))
+    assert all(m._lib.mla_uses_tensor_cores(C.byref(d), op) == 1 for op in range(5))
     assert m._lib.mla_uses_tensor_cores(C.byref(v2(m, dtype="fp32")), m.OP_DECODE) == 0
     assert m._lib.mla_uses_tensor_cores(C.byref(v2(m, n_h=64)), m.OP_DECODE) == 0
     assert m._lib.mla_uses_tensor_cores(C.byref(d), 9) == 0
