@@ -70,7 +70,23 @@ def parse():
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch kernels without programmatic dependent launch (mla_set_launch_overlap off)")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0, help="target seconds of oracle work")
+    ap.add_argument("--num-splits", type=int, default=0,
+                    help="mla_decode num_splits: 0 = automatic plan, S > 0 = each token row in min(S, its tiles) pieces")
+    ap.add_argument("--with-o-proj", action="store_true",
+                    help="add the output projection y = W_O o (mla_o_proj) to every step and time it on its own")
     return ap.parse_args()
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def cache_copies(cache_bytes):
+    """Copies of the latent cache the timed loop rotates through, so that a
+    step never finds its cache in L2 left by the step before: one when the cache
+    alone exceeds L2, else enough to cover twice the L2 size."""
+    if cache_bytes > L2_BYTES:
+        return 1
+    return min(8, -(-2 * L2_BYTES // cache_bytes))
 
 
 # ------------------------------------------------------------------ clocks --
@@ -196,9 +212,16 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("bench.py times the bf16 tensor-core workloads")
     x = synth.generate(w)
     W, cache_t, bt = upload(x, torch, dev)
-    cache = mla.Cache(cache_t, bt)
+    n_copies = cache_copies(cache_t.numel() * cache_t.element_size())
+    caches = [mla.Cache(cache_t, bt)] + [mla.Cache(cache_t.clone(), bt) for _ in range(n_copies - 1)]
     p = mla.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base, 0.0, w.dtype)
     T = w.T
+    HD = w.n_h * w.d_h
+    if args.with_o_proj:  # W_O ~ N(0, 1/(n_h d_h)) from its own seed, rounded to bf16
+        rng = np.random.Generator(np.random.PCG64(2000 + w.index))
+        W_O = rng.standard_normal((w.d, HD), dtype=np.float32) * np.float32(1.0 / math.sqrt(HD))
+        W["W_O"] = torch.from_numpy(synth.bf16_bits(W_O).view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((T, w.d), device=dev, dtype=torch.bfloat16)
     # two sets of the step's input and output buffers, so that the end-to-end
     # loop can copy the next step's inputs in while this step computes
     h_host = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16)
@@ -211,20 +234,25 @@ def run_ours(args, rank, world, local_rank):
     lse = torch.empty((T, w.n_h), device=dev, dtype=torch.float32)
     ws = {op: torch.empty(max(1, mla.workspace_size(p, op, w.B if op == mla.OP_DECODE else T, w.n_q)),
                           dtype=torch.uint8, device=dev)
-          for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ)}
+          for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ, mla.OP_O_PROJ)}
+    ws[mla.OP_DECODE] = torch.empty(max(1, mla.workspace_size(p, mla.OP_DECODE, w.B, w.n_q, mla.cache_capacity(caches[0]),
+                                                              args.num_splits)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)  # graph capture needs a non-default stream
     # the decode is bracketed by timing events in every timed step; "external"
     # makes them real event-record nodes when the step is captured in a graph
     ev_dec = [(torch.cuda.Event(enable_timing=True, external=True),
                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
+    ev_op = [(torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
 
     # the cache append and the query absorption are independent: the append
     # runs on a side stream, joined before the decode reads the cache
     side = torch.cuda.Stream(device=dev)
     ev_fork, ev_join = torch.cuda.Event(), torch.cuda.Event()
 
-    def step(i=None, b=0):
+    def step(i=None, b=0, c=None):
         x_ = bufs[b]
+        cache = caches[(i if c is None else c) % n_copies if (i is not None or c is not None) else 0]
         ev_fork.record(stream)
         side.wait_event(ev_fork)
         mla.mla_cache_append(p, x_["h"], W["W_DKV"], W["W_KR"], x_["sidx"], x_["pos"], cache,
@@ -235,10 +263,17 @@ def run_ours(args, rank, world, local_rank):
         stream.wait_event(ev_join)
         if i is not None:
             ev_dec[i][0].record(stream)
-        mla.mla_decode(p, q, cache, x_["sl"], w.n_q, o_lat, lse, ws=ws[mla.OP_DECODE], stream=stream)
+        mla.mla_decode(p, q, cache, x_["sl"], w.n_q, o_lat, lse, num_splits=args.num_splits, ws=ws[mla.OP_DECODE],
+                       stream=stream)
         if i is not None:
             ev_dec[i][1].record(stream)
         mla.mla_out_proj(p, o_lat, W["W_UV"], x_["o"], ws=ws[mla.OP_OUT_PROJ], stream=stream)
+        if args.with_o_proj:
+            if i is not None:
+                ev_op[i][0].record(stream)
+            mla.mla_o_proj(p, x_["o"], W["W_O"], y, ws=ws[mla.OP_O_PROJ], stream=stream)
+            if i is not None:
+                ev_op[i][1].record(stream)
 
     def barrier():
         if world > 1:
@@ -259,10 +294,11 @@ def run_ours(args, rank, world, local_rank):
     graph_1 = graph_k = None
     launches_k = 0
     if not args.eager:
-        graph_1, graph_k = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()], torch.cuda.CUDAGraph()
-        for b in range(2):
-            with torch.cuda.graph(graph_1[b], stream=stream):
-                step(b=b)
+        graph_1 = {(b, c): torch.cuda.CUDAGraph() for b in range(2) for c in range(n_copies)}
+        graph_k = torch.cuda.CUDAGraph()
+        for (b, c), g in graph_1.items():
+            with torch.cuda.graph(g, stream=stream):
+                step(b=b, c=c)
         n0 = mla.kernel_launches()
         with torch.cuda.graph(graph_k, stream=stream):
             for i in range(args.steps):
@@ -270,11 +306,11 @@ def run_ours(args, rank, world, local_rank):
         launches_k = mla.kernel_launches() - n0  # the kernels graph_k launches per replay
         torch.cuda.synchronize()
 
-    def one_step(b=0):
+    def one_step(b=0, c=0):
         if graph_1 is not None:
-            graph_1[b].replay()
+            graph_1[(b, c % n_copies)].replay()
         else:
-            step(b=b)
+            step(b=b, c=c)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -306,6 +342,7 @@ def run_ours(args, rank, world, local_rank):
     dec_list = [a.elapsed_time(b) for a, b in ev_dec]
     dec_ms = float(np.mean(dec_list))
     dec_pct = percentiles_us(dec_list)
+    op_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_op])) if args.with_o_proj else None
 
     # End to end through the public API: every step copies its inputs in from
     # pinned host memory and its output o back, inside the timed region. The
@@ -339,7 +376,7 @@ def run_ours(args, rank, world, local_rank):
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_out[b])  # o of step i - 2 has left set b
-            one_step(b)
+            one_step(b, i)
             ev_done[b].record(stream)
         with torch.cuda.stream(d2h_stream):
             d2h_stream.wait_event(ev_done[b])
@@ -357,87 +394,133 @@ def run_ours(args, rank, world, local_rank):
 
     step_ms = ms_total / args.steps
     if world > 1:
-        step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], dev)
+        step_ms, dec_ms, e2e_ms, op_ms = max_over_ranks([step_ms, dec_ms, e2e_ms, op_ms or 0.0], dev)
+        op_ms = op_ms if args.with_o_proj else None
     del graph_1, graph_k
     return {"step_ms": step_ms, "dec_ms": dec_ms, "dec_pct": dec_pct, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
             "launch_mode": ("eager" if args.eager else "cuda_graph") + ("" if args.no_overlap else "+overlap"),
-            "launches": launches, "clocks": clk.summary(), "x": x, "w": w,
+            "launches": launches, "clocks": clk.summary(), "x": x, "w": w, "op_ms": op_ms, "n_copies": n_copies,
             "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
 
 
 # ------------------------------------------------------ oracle (CPU) arm --
 
+def stratified_order(seq_lens):
+    """Sequences ordered so that every prefix spans the length distribution:
+    sorted by length, then taken alternately from the long and the short end
+    of ever finer halvings (a prefix is a fair sample of the batch)."""
+    idx = [int(b) for b in np.argsort(seq_lens, kind="stable")]
+    out, parts = [], [idx]
+    while parts:
+        nxt = []
+        for p_ in parts:
+            if not p_:
+                continue
+            m = len(p_) // 2
+            out.append(p_[m])
+            nxt += [p_[:m], p_[m + 1:]]
+        parts = nxt
+    return out
+
+
+def oracle_step(w, x, seqs):
+    """One step of the fp64 oracle over the token rows of `seqs`: append of
+    their new tokens, absorb, decode of all heads over the visible context,
+    W_UV readout. Returns (seconds, attended tokens)."""
+    import oracle as orc
+    po = orc.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base)
+    oc = orc.Cache(x.cache, x.block_table)
+    rows = [b * w.n_q + j for b in seqs for j in range(w.n_q)]
+    t0 = time.perf_counter()
+    orc.append_rows(po, x.h[rows], x.weights["W_DKV"], x.weights["W_KR"], x.positions[rows])
+    qb = orc.absorb_q(po, x.h[rows], x.weights["W_DQ"], x.weights["W_UQ"], x.weights["W_QR"],
+                      x.weights["W_UK"], x.positions[rows])
+    q = np.zeros((w.T, w.n_h, w.D))
+    q[rows] = qb
+    pairs = [(t, hh) for t in rows for hh in range(w.n_h)]
+    o_lat, _ = orc.decode(po, q, oc, x.seq_lens, w.n_q, pairs=pairs)
+    orc.out_proj(po, o_lat.reshape(len(rows), w.n_h, w.d_c), x.weights["W_UV"])
+    seconds = time.perf_counter() - t0
+    tokens = sum(int(x.seq_lens[b]) - w.n_q + 1 + j for b in seqs for j in range(w.n_q))
+    return seconds, tokens
+
+
 def oracle_sample(w, x, target_s):
-    """Time the fp64 oracle on a bounded sample of the workload: the whole step
-    for the token rows of a few sequences (append of their new tokens, absorb,
-    decode of all heads over their visible context, W_UV readout). Returns
-    (seconds per step extrapolated by attended-token work, sample text, cores)."""
+    """Time the fp64 oracle on a bounded sample of the workload: whole steps
+    over a growing, length-stratified set of sequences until about target_s of
+    work, the whole batch when it fits. Returns (seconds per step, scaled to the
+    whole batch by attended tokens when the sample is smaller, sample text,
+    cores)."""
     import oracle as orc
     cores = len(os.sched_getaffinity(0))
     orc.set_threads(cores)
-    po = orc.dims(w.d, w.n_h, w.d_h, w.d_c, w.d_cq, w.d_r, w.rope_base)
-    oc = orc.Cache(x.cache, x.block_table)
     work_total = synth.algorithmic_work(w, x.seq_lens)["tokens_attended"]
-    order = np.argsort(x.seq_lens)  # shortest first, grow until the target time
-    done_tokens, seconds, seqs = 0, 0.0, 0
-    t_start = time.perf_counter()
-    for b in order:
-        b = int(b)
-        rows = list(range(b * w.n_q, (b + 1) * w.n_q))
-        t0 = time.perf_counter()
-        orc.append_rows(po, x.h[rows], x.weights["W_DKV"], x.weights["W_KR"], x.positions[rows])
-        qb = orc.absorb_q(po, x.h[rows], x.weights["W_DQ"], x.weights["W_UQ"], x.weights["W_QR"],
-                          x.weights["W_UK"], x.positions[rows])
-        q = np.zeros((w.T, w.n_h, w.D))
-        q[rows] = qb
-        pairs = [(t, hh) for t in rows for hh in range(w.n_h)]
-        o_lat, _ = orc.decode(po, q, oc, x.seq_lens, w.n_q, pairs=pairs)
-        orc.out_proj(po, o_lat.reshape(len(rows), w.n_h, w.d_c), x.weights["W_UV"])
-        seconds += time.perf_counter() - t0
-        done_tokens += sum(int(x.seq_lens[b]) - w.n_q + 1 + j for j in range(w.n_q))
-        seqs += 1
-        if time.perf_counter() - t_start > target_s:
-            break
-    per_step = seconds * work_total / max(1, done_tokens)
-    sample = (f"full step (append, absorb, decode over all {w.n_h} heads, W_UV readout) for {seqs} of "
-              f"{w.B} sequences ({done_tokens} attended tokens of {work_total}); time scaled to the whole "
-              f"batch by attended tokens")
+    order = stratified_order(x.seq_lens)
+    seconds, tokens, n = 0.0, 0, 0
+    chunk = max(1, len(order) // 16)
+    while n < len(order) and (n == 0 or seconds < target_s):
+        s, t = oracle_step(w, x, order[n:n + chunk])
+        seconds, tokens, n = seconds + s, tokens + t, min(len(order), n + chunk)
+    whole = n == len(order)
+    per_step = seconds if whole else seconds * work_total / max(1, tokens)
+    sample = (f"full step (append, absorb, decode over all {w.n_h} heads, W_UV readout) for {n} of {w.B} "
+              f"sequences ({tokens} attended tokens of {work_total})"
+              + ("; the whole batch, no scaling" if whole else
+                 "; length-stratified sample, time scaled to the whole batch by attended tokens"))
     return per_step, sample, cores
 
 
 def run_reference(args, rank, world):
+    """The oracle arm: every timed step runs the fp64 oracle over the whole
+    batch (all sequences, all heads), so that steps x ms_per_step is the time
+    the arm really took. Warm-up steps run one sequence each (they only page
+    the oracle and its inputs in)."""
+    import oracle as orc
     w = synth.WORKLOADS[args.workload]
     x = synth.generate(w)
-    per_step_s = []
-    sample_text, cores = "", 0
-    for _ in range(max(1, args.warmup // 3)):
-        oracle_sample(w, x, target_s=min(3.0, args.cpu_sample_s))
-    for _ in range(args.steps):
-        s, sample_text, cores = oracle_sample(w, x, target_s=args.cpu_sample_s / max(1, args.steps))
-        per_step_s.append(s)
+    cores = len(os.sched_getaffinity(0))
+    orc.set_threads(cores)
+    order = stratified_order(x.seq_lens)
+    for _ in range(args.warmup):
+        oracle_step(w, x, order[:1])
+    per_step_s = [oracle_step(w, x, order)[0] for _ in range(args.steps)]
     us = float(np.mean(per_step_s) * 1e6)
     work = synth.algorithmic_work(w, x.seq_lens)
+    sample = (f"whole batch every step: full step (append, absorb, decode over all {w.n_h} heads, W_UV readout) "
+              f"for all {w.B} sequences ({work['tokens_attended']} attended tokens); warm-up steps: one sequence")
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": "µs/step", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, args.gpus, x), "gpu_launches": 0,
-        "cpu_baseline": {"value": us, "unit": "µs/step", "cores": cores, "kind": "oracle",
-                         "sample": sample_text},
+        "config": config_of(w, args.gpus, x, None, args), "gpu_launches": 0,
+        "cpu_baseline": {"value": us, "unit": "µs/step", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": us, "unit": "µs/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "cache_gbs": work["cache_bytes"] / (us * 1e-6) / 1e9,
     }
     print(json.dumps(line))
 
 
-def config_of(w, n, x):
+def config_of(w, n, x, n_copies=None, args=None):
     L = x.seq_lens
+    cache_bytes = int(x.cache.nbytes)
+    if n_copies is None:
+        n_copies = cache_copies(cache_bytes)
+    l2 = ("no flush: the latent cache alone ({:.1f} MB) exceeds the 126 MB L2 (inputs larger than L2)".format(
+        cache_bytes / 1e6) if n_copies == 1 else
+        "the timed steps rotate through {} copies of the {:.1f} MB latent cache ({:.0f} MB > 2 x L2), so no step "
+        "finds its cache in L2".format(n_copies, cache_bytes / 1e6, n_copies * cache_bytes / 1e6))
     return {"workload": w.name, "description": w.note, "batch": w.B, "n_q": w.n_q,
             "seq_len_min": int(L.min()), "seq_len_max": int(L.max()), "seq_len_mean": float(L.mean()),
             "paged": w.paged, "block_size": w.block_size if w.paged else None,
             "dims": {"d": w.d, "n_h": w.n_h, "d_h": w.d_h, "d_c": w.d_c, "d_cq": w.d_cq, "d_r": w.d_r},
-            "parallelism": f"replicas{n}", "seed": 1000 + w.index,
-            "l2": "no flush: latent cache and weights each exceed the 126 MB L2 (inputs larger than L2)"}
+            "parallelism": f"replicas{n}", "seed": 1000 + w.index, "l2": l2,
+            "num_splits": 0 if args is None else args.num_splits,
+            "step": "append + absorb + decode + W_UV readout" + (" + W_O projection" if args is not None and
+                                                                 args.with_o_proj else "")}
+
+
+def HD_of(w):
+    return w.n_h * w.d_h
 
 
 def main():
@@ -492,7 +575,8 @@ def main():
     line = {
         "metric": METRIC, "value": us, "unit": "µs/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world, x),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, world, x, r["n_copies"], args),
         "decode_us": r["dec_ms"] * 1e3, "decode_us_p10_p50_p90": r["dec_pct"], "cache_gbs": cache_gbs,
         "tflops": tflops,
         "tokens_per_s": world * w.T / (r["step_ms"] * 1e-3),
@@ -500,6 +584,10 @@ def main():
         "e2e": {"value": r["e2e_ms"] * 1e3, "unit": "µs/step", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
+        **({"o_proj": {"us": r["op_ms"] * 1e3, "weight_bytes": w.d * HD_of(w) * 2,
+                       "gbs": w.d * HD_of(w) * 2 / (r["op_ms"] * 1e-3) / 1e9,
+                       "frac": (w.d * HD_of(w) * 2 / (peaks["hbm_gbs"] * 1e9)) / (r["op_ms"] * 1e-3),
+                       "peak_gbs": peaks["hbm_gbs"]}} if r["op_ms"] is not None else {}),
         "tensor_core_decode": r["tc"],
         "clocks": r["clocks"],
     }

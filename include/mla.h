@@ -132,9 +132,15 @@ mla_status mla_absorb_q(const mla_dims *dims, const void *h, const void *W_DQ, c
  *   q [B*n_q][n_h][D]   seq_lens [B] int32 device
  *   o_lat (output) [B*n_q][n_h][d_c] storage dtype
  *   lse (output, may be NULL) [B*n_q][n_h] float32 (natural log)
- * num_splits: 0 = automatic split-KV planning; the tensor-core path always
- * balances the concatenated KV tiles of all sequences over the GPU and merges
- * split sequences with a log-sum-exp combine, so only 0 is accepted there.
+ * num_splits (split-KV): 0 = automatic: the tensor-core path concatenates the
+ * 256-token KV tiles of all token rows, cuts that line into one equal share
+ * per pair of SMs, and merges every row cut by a share boundary with a
+ * log-sum-exp combine. S > 0 = forced: every token row is cut into
+ * min(S, its tiles) pieces of near-equal tile counts (S = 1: no split), each
+ * pair of SMs takes the pieces that start in its equal share of the tile line,
+ * and rows of more than one piece are merged by the same combine. The
+ * CUDA-core path (fp32 or other dims) never splits and ignores S. Results
+ * agree within rounding for every S.
  * seq_lens[b] < n_q or beyond the cache capacity raises MLA_ERR_DEVICE_DATA
  * and that sequence's outputs are left unwritten. */
 mla_status mla_decode(const mla_dims *dims, const void *q, const mla_cache *cache,
@@ -150,8 +156,9 @@ mla_status mla_decode(const mla_dims *dims, const void *q, const mla_cache *cach
  *   35 MB, reserved when the library's device code is loaded. Larger calls
  *   return MLA_ERR_UNSUPPORTED with the reason in mla_last_error_message().
  *   The library allocates nothing.
- *   First call on each device looks up that device's copy of the array
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   The first call on each device, and the first call after a device reset,
+ *   looks up that device's copy of the array (cudaGetSymbolAddress); make that
+ *   call before any stream capture.
  *   Nothing in the scratch needs to start at zero: every call writes each
  *   byte it later reads.
  *   The scratch is shared by all callers in the process: calls that can
@@ -177,11 +184,14 @@ mla_status mla_o_proj(const mla_dims *dims, const void *o, const void *W_O, int3
                       size_t ws_bytes, void *stream);
 
 /* Scratch size in bytes for one call of `op` (MLA_OP_*). `rows` is T for
- * append/absorb/out_proj and B for decode; n_q and max_seq_len are used by
- * decode only (max_seq_len may be 0 for the tensor-core path). */
+ * append/absorb/out_proj/o_proj and B for decode; n_q, max_seq_len and
+ * num_splits are used by decode only. max_seq_len bounds the tiles of a row
+ * for forced splits (0 = unknown: the size then covers num_splits pieces for
+ * every row); mla_decode itself requires the size for max_seq_len = the
+ * cache's capacity (max_len, or max_blocks_per_seq * block_size). */
 enum { MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3, MLA_OP_O_PROJ = 4 };
 size_t mla_workspace_size(const mla_dims *dims, int32_t op, int32_t rows, int32_t n_q,
-                          int64_t max_seq_len);
+                          int64_t max_seq_len, int32_t num_splits);
 
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns MLA_OK, MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_DATA or MLA_ERR_CUDA. */

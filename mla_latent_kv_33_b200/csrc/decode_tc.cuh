@@ -52,6 +52,9 @@
 //    that k_combine merges with a log-sum-exp. (Merging them in the epilogue
 //    of the CTA that finishes a row's last piece measured slower: the merge
 //    then runs on one SM's bandwidth, on that cluster's critical path.)
+//    With a forced split count S (Params::splits > 0) every row is instead
+//    cut into min(S, its tiles) pieces of near-equal tile counts, and each
+//    cluster takes the pieces that start in its equal share of the tile line.
 //  * Rows past a sequence's end: 64-row blocks wholly past it are loaded at
 //    an out-of-range coordinate (TMA zero fill); the one partially valid block
 //    has its value rows past the end zeroed in shared memory before its PV
@@ -96,7 +99,7 @@ constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(NUM_BARS * 8 <= MISC_RED, "barriers overlap the exchange arrays");
 static_assert(SMEM_BYTES <= 232448, "decode shared memory budget");
 static_assert(OFF_BIG % 1024 == 0 && OFF_SMALL % 1024 == 0, "128-byte swizzle alignment");
-constexpr int MAX_UNITS = (NBIG * BIG + SMALL) / 4 - 1;  // plan scratch aliases the ring
+constexpr int MAX_UNITS = (NBIG * BIG + SMALL) / 8 - 1;  // plan scratch (two ints per row) aliases the ring
 constexpr int S_COL = 256;  // TMEM: O at [0,256); scores, then P over them, at [256 + 128 b, +128)
 constexpr uint32_t IDESC_S = idesc_bf16(128, 256, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
@@ -123,8 +126,15 @@ struct Params {
   float *lse;
   float *part_o;    // [slots][128][512]
   float *part_lse;  // [slots][128]
-  int32_t *plan;    // [0] = W, [1] = Qt, [2..] = tile offsets [BJ + 1]
+  // [0] = W (visible tiles), [1] = Qt (tiles per cluster, automatic plan), [2] = splits,
+  // [3 ..] tile offsets of the rows [BJ + 1], then (splits > 0) piece offsets [BJ + 1]
+  int32_t *plan;
+  int32_t splits;   // 0: automatic plan; S > 0: every row in min(S, tiles) pieces
 };
+
+// Offsets of the plan arrays in Params::plan.
+__host__ __device__ constexpr int plan_tiles(int) { return 3; }
+__host__ __device__ constexpr int plan_pieces(int BJ) { return 4 + BJ; }
 
 // Tiles visible to unit bj (token row); -1 if its sequence length is invalid.
 __device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out) {
@@ -171,14 +181,28 @@ __device__ __forceinline__ void tile_rows(const Params &p, int b, int64_t t0, in
 
 struct Piece {
   int bj, t_begin, t_end, vis, nt;
-  bool single;
-  int slot;
-  int k0, k1;  // clusters holding the first and last piece of the row (slots bj + k0 .. bj + k1)
+  bool single;  // the row's only piece: o_lat and lse are written in place
+  int slot;     // split partial slot of this piece (when not single)
 };
 
-// Iterates the pieces of this cluster's tile range in order.
+__device__ __forceinline__ int split_pieces(int S, int nt) { return nt < S ? nt : S; }
+
+// End (row-relative tile) of the forced-split piece holding tile r of a row
+// with nt tiles cut into sp pieces (piece q covers [q nt / sp, (q + 1) nt / sp)),
+// and that piece's index.
+__device__ __forceinline__ int split_piece_of(int r, int nt, int sp, int *end) {
+  const int q = static_cast<int>((static_cast<int64_t>(r + 1) * sp - 1) / nt);
+  *end = static_cast<int>(static_cast<int64_t>(q + 1) * nt / sp);
+  return q;
+}
+
+// Iterates the pieces of this cluster's tile range in order. Automatic plan:
+// pieces are cut by row ends and cluster boundaries, and the split slot of a
+// row's piece in cluster k is bj + k (a cluster holds at most one piece of a
+// row that continues into another cluster). Forced splits: pieces are also cut
+// at the row's piece boundaries, and the slot is the piece's global index.
 struct PieceIter {
-  int g, gend, bj, off, Qt, k;
+  int g, gend, bj, off, poff, Qt, k, S;
   __device__ bool next(const Params &p, Piece &pc) {
     while (g < gend) {
       int vis;
@@ -186,6 +210,7 @@ struct PieceIter {
       if (nt < 0) nt = 0;
       if (nt == 0 || off + nt <= g) {
         off += nt;
+        poff += S ? split_pieces(S, nt) : 0;
         ++bj;
         continue;
       }
@@ -193,11 +218,25 @@ struct PieceIter {
       pc.vis = vis;
       pc.nt = nt;
       pc.t_begin = g - off;
+      if (S) {
+        const int sp = split_pieces(S, nt);
+        int pend;
+        const int q = split_piece_of(g - off, nt, sp, &pend);
+        const int e = min(gend, off + pend);
+        pc.t_end = e - off;
+        pc.single = sp == 1;
+        pc.slot = poff + q;
+        g = e;
+        if (e == off + nt) {
+          off += nt;
+          poff += sp;
+          ++bj;
+        }
+        return true;
+      }
       const int e = min(gend, off + nt);
       pc.t_end = e - off;
-      pc.k0 = off / Qt;
-      pc.k1 = (off + nt - 1) / Qt;
-      pc.single = pc.k0 == pc.k1;
+      pc.single = off / Qt == (off + nt - 1) / Qt;
       pc.slot = bj + k;
       g = e;
       off += nt;
@@ -207,6 +246,61 @@ struct PieceIter {
     return false;
   }
 };
+
+// In-place exclusive prefix sum of a[0 .. n) by the whole block; returns the
+// total to every thread. wtot: NUM_THREADS / 32 ints of shared memory.
+template <int NT>
+__device__ int block_exclusive_scan(int *a, int n, int *wtot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = (n + NT - 1) / NT;
+  const int lo = min(n, static_cast<int>(threadIdx.x) * per), hi = min(n, lo + per);
+  int sum = 0;
+  for (int u = lo; u < hi; ++u) sum += a[u];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  int base = 0, total = 0;
+  for (int w = 0; w < NT / 32; ++w) {
+    if (w < warp) base += wtot[w];
+    total += wtot[w];
+  }
+  int run = base + incl - sum;
+  for (int u = lo; u < hi; ++u) {
+    const int v = a[u];
+    a[u] = run;
+    run += v;
+  }
+  __syncthreads();
+  return total;
+}
+
+// Row holding tile G of the tile line (prefix[] = exclusive tile offsets of
+// the BJ rows, G < W): the last row whose offset is <= G, which is never empty.
+__device__ __forceinline__ int row_of_tile(const int *prefix, int BJ, int G) {
+  int lo = 0, hi = BJ - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= G) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// First forced-split piece boundary at or after tile G of the tile line.
+__device__ __forceinline__ int snap_to_piece(const int *prefix, int BJ, int W, int S, int G) {
+  if (G >= W) return W;
+  const int u = row_of_tile(prefix, BJ, G);
+  const int nt = (u + 1 < BJ ? prefix[u + 1] : W) - prefix[u];
+  const int sp = split_pieces(S, nt), r = G - prefix[u];
+  int pend;
+  const int q = split_piece_of(r, nt, sp, &pend);
+  const int pbeg = static_cast<int>(static_cast<int64_t>(q) * nt / sp);
+  return pbeg == r ? G : prefix[u] + pend;
+}
 
 // The value chunk of tile ti that needs zeroed rows (holds the last visible
 // token but not 64 visible tokens), or -1.
@@ -242,7 +336,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   int *ints = reinterpret_cast<int *>(misc + MISC_INTS);
   volatile int *abort_flag = ints + 0;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ints + 1);
-  int *plan_s = ints + 2;  // W, Qt, bj_first, off_first
+  int *plan_s = ints + 2;  // g0, g1, Qt, first row, its tile offset, its piece offset
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
@@ -275,9 +369,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   // workspace: only once the previous kernel on the stream has finished
   griddep_wait();
 
-  // ---- plan: tiles per unit, prefix sums, this cluster's first unit ----
+  // ---- plan: tiles (and forced pieces) per unit, prefix sums, this cluster's range ----
   const int BJ = p.B * p.n_q;
-  int *scratch = reinterpret_cast<int *>(smem + OFF_BIG);
+  const int S = p.splits;
+  int *tiles = reinterpret_cast<int *>(smem + OFF_BIG);  // [BJ], then (S > 0) pieces [BJ]
+  int *pieces = tiles + BJ;
   for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
     int vis;
     int nt = unit_tiles(p, u, &vis);
@@ -285,56 +381,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       if (blockIdx.x == 0 && (u % p.n_q) == 0) dev_error(MLA_DEVERR_DATA);
       nt = 0;
     }
-    scratch[u] = nt;
+    tiles[u] = nt;
+    if (S) pieces[u] = split_pieces(S, nt);
   }
   __syncthreads();
   {
-    const int per = (BJ + NUM_THREADS - 1) / NUM_THREADS;
-    const int lo = threadIdx.x * per, hi = min(BJ, lo + per);
-    int sum = 0;
-    for (int u = lo; u < hi; ++u) sum += scratch[u];
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
     __shared__ int warp_tot[NUM_THREADS / 32];
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    int run = base + incl - sum;
-    for (int u = lo; u < hi; ++u) {
-      const int nt = scratch[u];
-      scratch[u] = run;
-      run += nt;
-    }
-    if (threadIdx.x == NUM_THREADS - 1) {
-      int W = 0;
-      for (int w = 0; w < NUM_THREADS / 32; ++w) W += warp_tot[w];
-      plan_s[0] = W;
-      plan_s[1] = max(1, (W + nclusters - 1) / nclusters);
-      plan_s[2] = BJ;
-      plan_s[3] = W;
-    }
-    __syncthreads();
-    const int W = plan_s[0], Qt = plan_s[1];
-    const int g0 = cluster * Qt;
-    for (int u = lo; u < hi; ++u) {
-      const int a = scratch[u];
-      const int e = (u + 1 < BJ) ? scratch[u + 1] : W;
-      if (a <= g0 && g0 < e) {
-        plan_s[2] = u;
-        plan_s[3] = a;
+    const int W = block_exclusive_scan<NUM_THREADS>(tiles, BJ, warp_tot);
+    const int P = S ? block_exclusive_scan<NUM_THREADS>(pieces, BJ, warp_tot) : 0;
+    if (threadIdx.x == 0) {
+      int g0, g1, Qt = 0;
+      if (S == 0) {
+        Qt = max(1, (W + nclusters - 1) / nclusters);
+        g0 = min(W, cluster * Qt);
+        g1 = min(W, (cluster + 1) * Qt);
+      } else {
+        const auto share = [&](int c) {
+          return static_cast<int>((static_cast<int64_t>(c) * W + nclusters - 1) / nclusters);
+        };
+        g0 = snap_to_piece(tiles, BJ, W, S, share(cluster));
+        g1 = snap_to_piece(tiles, BJ, W, S, share(cluster + 1));
       }
+      const int u0 = g0 < W ? row_of_tile(tiles, BJ, g0) : BJ;
+      plan_s[0] = g0;
+      plan_s[1] = g1;
+      plan_s[2] = Qt;
+      plan_s[3] = u0;
+      plan_s[4] = u0 < BJ ? tiles[u0] : W;
+      plan_s[5] = S && u0 < BJ ? pieces[u0] : 0;
     }
-    if (blockIdx.x == 0) {
-      for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) p.plan[2 + u] = scratch[u];
+    if (blockIdx.x == 0) {  // the layout k_combine reads
+      for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
+        p.plan[plan_tiles(BJ) + u] = tiles[u];
+        if (S) p.plan[plan_pieces(BJ) + u] = pieces[u];
+      }
       if (threadIdx.x == 0) {
         p.plan[0] = W;
-        p.plan[1] = Qt;
-        p.plan[2 + BJ] = W;
+        p.plan[1] = S == 0 ? max(1, (W + nclusters - 1) / nclusters) : 0;
+        p.plan[2] = S;
+        p.plan[plan_tiles(BJ) + BJ] = W;
+        if (S) p.plan[plan_pieces(BJ) + BJ] = P;
       }
     }
   }
@@ -343,14 +429,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   cluster_sync_all();  // peer barriers initialised, TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int W = plan_s[0], Qt = plan_s[1];
   PieceIter it0;
-  it0.g = min(W, cluster * Qt);
-  it0.gend = min(W, (cluster + 1) * Qt);
-  it0.bj = plan_s[2];
-  it0.off = plan_s[3];
-  it0.Qt = Qt;
+  it0.g = plan_s[0];
+  it0.gend = plan_s[1];
+  it0.Qt = max(1, plan_s[2]);
+  it0.bj = plan_s[3];
+  it0.off = plan_s[4];
+  it0.poff = plan_s[5];
   it0.k = cluster;
+  it0.S = S;
 
   if (warp < NUM_PRODUCERS) {
     // --------------------------------------------------------- ring producers
@@ -764,14 +851,22 @@ __global__ void __launch_bounds__(128) k_combine(Params p) {
   const int bj = blockIdx.x / COMBINE_BLOCKS_PER_ROW;
   const int head = 4 * (blockIdx.x % COMBINE_BLOCKS_PER_ROW) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const int a = p.plan[2 + bj], e = p.plan[3 + bj], Qt = p.plan[1];
-  if (e <= a) return;
-  const int k0 = a / Qt, k1 = (e - 1) / Qt;
-  if (k0 == k1) return;
-  const int np = k1 - k0 + 1;
-  const float *pl = p.part_lse + static_cast<int64_t>(bj + k0) * HEADS + head;
+  const int BJ = p.B * p.n_q;
+  int first, np;
+  if (p.plan[2] == 0) {  // automatic plan: the row's pieces are its clusters k0 .. k1, slots bj + k
+    const int a = p.plan[plan_tiles(BJ) + bj], e = p.plan[plan_tiles(BJ) + bj + 1], Qt = p.plan[1];
+    if (e <= a) return;
+    const int k0 = a / Qt, k1 = (e - 1) / Qt;
+    first = bj + k0;
+    np = k1 - k0 + 1;
+  } else {  // forced splits: the row's pieces are slots piece_off[bj] ..
+    first = p.plan[plan_pieces(BJ) + bj];
+    np = p.plan[plan_pieces(BJ) + bj + 1] - first;
+  }
+  if (np <= 1) return;
+  const float *pl = p.part_lse + static_cast<int64_t>(first) * HEADS + head;
   const float4 *po =
-      reinterpret_cast<const float4 *>(p.part_o + (static_cast<int64_t>(bj + k0) * HEADS + head) * DC) + lane;
+      reinterpret_cast<const float4 *>(p.part_o + (static_cast<int64_t>(first) * HEADS + head) * DC) + lane;
   constexpr int64_t PIECE4 = static_cast<int64_t>(HEADS) * DC / 4;  // float4 stride between pieces
   float M = -INFINITY, Z = 0.f;
   float4 acc[4];
@@ -832,13 +927,24 @@ __global__ void __launch_bounds__(128) k_combine(Params p) {
 
 }  // namespace dec
 
-// Workspace: plan (W, Qt, BJ + 1 offsets), then split partials for at most
-// BJ + clusters slots.
-inline size_t decode_plan_bytes(size_t BJ) { return ((BJ + 3) * sizeof(int32_t) + 255) & ~size_t(255); }
-inline size_t decode_tc_ws(int B, int n_q, int sms) {
+// Workspace: the plan (3 words, tile offsets and piece offsets of the BJ + 1
+// row boundaries), then fp32 split partials. Slots: at most BJ + clusters for
+// the automatic plan; for S forced splits at most BJ * min(S, tiles of the
+// longest row), max_seq_len (0 = unknown) bounding the tiles.
+constexpr size_t decode_plan_bytes(size_t BJ) { return ((2 * BJ + 5) * sizeof(int32_t) + 255) & ~size_t(255); }
+inline size_t decode_tc_slots(int B, int n_q, int sms, int splits, int64_t max_seq_len) {
   const size_t BJ = static_cast<size_t>(B) * n_q;
-  const size_t clusters = static_cast<size_t>(sms / 2);
-  const size_t slots = BJ + clusters;
+  size_t slots = BJ + static_cast<size_t>(sms / 2);
+  if (splits > 0) {
+    int64_t per_row = splits;
+    if (max_seq_len > 0) per_row = std::min<int64_t>(per_row, (max_seq_len + dec::TILE - 1) / dec::TILE);
+    slots = std::max(slots, BJ * static_cast<size_t>(per_row));
+  }
+  return slots;
+}
+inline size_t decode_tc_ws(int B, int n_q, int sms, int splits = 0, int64_t max_seq_len = 0) {
+  const size_t BJ = static_cast<size_t>(B) * n_q;
+  const size_t slots = decode_tc_slots(B, n_q, sms, splits, max_seq_len);
   return decode_plan_bytes(BJ) + slots * dec::HEADS * dec::DC * sizeof(float) + slots * dec::HEADS * sizeof(float);
 }
 

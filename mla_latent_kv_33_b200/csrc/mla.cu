@@ -570,10 +570,23 @@ mla_status tc_o_proj(const mla_dims *d, const void *o, const void *W_O, int T, v
 
 // Clusters of two CTAs that can be resident at once (a pair must share a GPC,
 // so this can be below SMs / 2). The persistent decode grid uses exactly this
-// many so that no cluster waits for a second wave.
+// many so that no cluster waits for a second wave. Occupancy is a property of
+// the device, so the count is cached per device ordinal; it never exceeds
+// half of that device's SMs, which is what decode_tc_ws() sizes the split
+// partials for.
+constexpr int MAX_DEVICES = 64;
+std::atomic<int> g_decode_clusters[MAX_DEVICES];
+
 int decode_clusters(int sms) {
-  static int cached = 0;
-  if (cached > 0) return cached;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  if (dev >= 0 && dev < MAX_DEVICES) {
+    const int c = g_decode_clusters[dev].load(std::memory_order_acquire);
+    if (c > 0) return std::min(c, sms / 2);
+  }
   namespace D = mla::dec;
   cudaFuncSetAttribute(D::k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES);
   cudaLaunchConfig_t cfg = {};
@@ -592,12 +605,18 @@ int decode_clusters(int sms) {
     cudaGetLastError();
     n = sms / 2;
   }
-  cached = std::min(n, sms / 2);
-  return cached;
+  n = std::max(1, std::min(n, sms / 2));
+  if (dev >= 0 && dev < MAX_DEVICES) g_decode_clusters[dev].store(n, std::memory_order_release);
+  return n;
+}
+
+// Longest sequence the cache can hold (bounds the tiles of a row).
+int64_t cache_capacity(const mla_cache *c) {
+  return c->paged ? static_cast<int64_t>(c->max_blocks_per_seq) * c->block_size : c->max_len;
 }
 
 mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int B, int n_q,
-                     void *o_lat, float *lse, void *ws, size_t ws_bytes, cudaStream_t st) {
+                     void *o_lat, float *lse, int num_splits, void *ws, size_t ws_bytes, cudaStream_t st) {
   namespace D = mla::dec;
   const int BJ = B * n_q;
   if (BJ > D::MAX_UNITS) return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode supports B*n_q <= %d", D::MAX_UNITS);
@@ -607,7 +626,8 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   if (rows >= 0x7fff0000LL) return fail(MLA_ERR_UNSUPPORTED, "cache has too many rows for 32-bit TMA coordinates");
   const int sms = sm_count();
   const int nclusters = decode_clusters(sms);
-  if (ws_bytes < mla::decode_tc_ws(B, n_q, sms)) return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
+  if (ws_bytes < mla::decode_tc_ws(B, n_q, sms, num_splits, cache_capacity(c)))
+    return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
 
   // Views of q and the cache (rows of 576 bf16 = 1152 bytes):
   //   q:        (64 cols, row, 9 chunks of 128 B)        box (64, 64 heads, 9)
@@ -650,8 +670,9 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.o_lat = static_cast<__nv_bfloat16 *>(o_lat);
   p.lse = lse;
+  p.splits = num_splits;
   const size_t plan_bytes = mla::decode_plan_bytes(BJ);
-  const size_t slots = static_cast<size_t>(BJ) + nclusters;
+  const size_t slots = mla::decode_tc_slots(B, n_q, sms, num_splits, cache_capacity(c));
   p.plan = static_cast<int32_t *>(ws);
   p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan_bytes);
   p.part_lse = p.part_o + slots * D::HEADS * D::DC;
@@ -681,10 +702,10 @@ namespace {
 
 constexpr int32_t NOALLOC_MAX_ROWS = 64;
 constexpr int32_t NOALLOC_MAX_CLUSTERS = 74;
-// plan (rows + 3 ints, 256-byte aligned), then fp32 partials [slots][128][512]
-// and [slots][128] for slots = rows + clusters (the decode workspace layout)
+// the decode workspace layout: the plan, then fp32 partials [slots][128][512]
+// and [slots][128] for slots = rows + clusters (automatic plan)
 constexpr size_t NOALLOC_BYTES =
-    ((static_cast<size_t>(NOALLOC_MAX_ROWS) + 3) * sizeof(int32_t) + 255) / 256 * 256 +
+    mla::decode_plan_bytes(NOALLOC_MAX_ROWS) +
     static_cast<size_t>(NOALLOC_MAX_ROWS + NOALLOC_MAX_CLUSTERS) * mla::dec::HEADS * (mla::dec::DC + 1) * sizeof(float);
 
 }  // namespace
@@ -693,25 +714,40 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
 namespace {
 
-constexpr int NOALLOC_MAX_DEVICES = 64;
-
-// Address of this device's copy of g_noalloc_scratch, looked up on the first
-// call from each device.
+// Address of the current device's copy of g_noalloc_scratch. It is looked up
+// with cudaGetSymbolAddress on the first call in each CUDA context of a
+// device and cached with that context's handle: after a device reset the
+// library's device code is loaded again, possibly elsewhere, in a new
+// context, and the next call looks the address up again.
 mla_status noalloc_scratch(void **ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "mla_decode_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES)
-    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc: device ordinal %d >= %d", dev, NOALLOC_MAX_DEVICES);
+  if (dev < 0 || dev >= MAX_DEVICES)
+    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc: device ordinal %d >= %d", dev, MAX_DEVICES);
+  // the current context (runtime calls make the device's primary context current)
+  static PFN_cuCtxGetCurrent_v4000 ctx_current = [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      fn = nullptr;
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }();
+  CUcontext ctx = nullptr;
+  if (ctx_current == nullptr || ctx_current(&ctx) != CUDA_SUCCESS)
+    return fail(MLA_ERR_CUDA, "mla_decode_noalloc: cannot query the current CUDA context");
   static std::mutex mu;
-  static void *addr[NOALLOC_MAX_DEVICES] = {};
+  static void *addr[MAX_DEVICES] = {};
+  static CUcontext addr_ctx[MAX_DEVICES] = {};
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || addr_ctx[dev] != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess)
       return fail(MLA_ERR_CUDA, "mla_decode_noalloc: cudaGetSymbolAddress of the scratch: %s", cudaGetErrorString(e));
     addr[dev] = p;
+    addr_ctx[dev] = ctx;
   }
   *ptr = addr[dev];
   return MLA_OK;
@@ -752,14 +788,15 @@ int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   return (op >= MLA_OP_APPEND && op <= MLA_OP_O_PROJ) ? 1 : 0;
 }
 
-size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len) {
-  (void)max_seq_len;
-  if (d == nullptr || rows <= 0) return 0;
+size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len,
+                          int32_t num_splits) {
+  if (d == nullptr || rows <= 0 || num_splits < 0) return 0;
   const bool tc = tc_geometry(d);
   switch (op) {
     case MLA_OP_APPEND: return tc ? tc_append_ws(d, rows) : simt_append_ws(d, rows);
     case MLA_OP_ABSORB: return tc ? tc_absorb_ws(d, rows) : simt_absorb_ws(d, rows);
-    case MLA_OP_DECODE: return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count()) : 0;
+    case MLA_OP_DECODE:
+      return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count(), num_splits, max_seq_len) : 0;
     case MLA_OP_OUT_PROJ: return tc ? tc_out_proj_ws(d, rows) : simt_out_proj_ws(d, rows);
     case MLA_OP_O_PROJ: return tc ? tc_o_proj_ws(d, rows) : simt_o_proj_ws(d, rows);
   }
@@ -790,7 +827,7 @@ mla_status mla_cache_append(const mla_dims *d, const void *h, const void *W_DKV,
   if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(W_KR))
     return fail(MLA_ERR_INVALID_ARG, "append: h and weights must be 16-byte aligned");
   if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
-  const size_t need = mla_workspace_size(d, MLA_OP_APPEND, T, 1, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_APPEND, T, 1, 0, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "append needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_geometry(d)) return tc_append(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, st);
@@ -810,7 +847,7 @@ mla_status mla_absorb_q(const mla_dims *d, const void *h, const void *W_DQ, cons
   if (!aligned16(h) || !aligned16(W_DQ) || !aligned16(W_UQ) || !aligned16(W_QR) || !aligned16(W_UK) ||
       !aligned16(q))
     return fail(MLA_ERR_INVALID_ARG, "absorb: tensors must be 16-byte aligned");
-  const size_t need = mla_workspace_size(d, MLA_OP_ABSORB, T, 1, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_ABSORB, T, 1, 0, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "absorb needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_geometry(d)) return tc_absorb(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, st);
@@ -830,14 +867,10 @@ mla_status mla_decode(const mla_dims *d, const void *q, const mla_cache *c, cons
   if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
   if (B > c->num_seqs) return fail(MLA_ERR_INVALID_ARG, "B exceeds cache->num_seqs");
   if (num_splits < 0) return fail(MLA_ERR_INVALID_ARG, "num_splits must be >= 0");
-  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, cache_capacity(c), num_splits);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "decode needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tc_geometry(d)) {
-    if (num_splits != 0)
-      return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode plans its own splits: pass num_splits = 0");
-    return decode_tc(d, q, c, seq_lens, B, n_q, o_lat, lse, ws, ws_bytes, st);
-  }
+  if (tc_geometry(d)) return decode_tc(d, q, c, seq_lens, B, n_q, o_lat, lse, num_splits, ws, ws_bytes, st);
   if (d->dtype == MLA_BF16) return simt_decode<__nv_bfloat16>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
   return simt_decode<float>(d, q, c, seq_lens, B, n_q, o_lat, lse, st);
 }
@@ -850,7 +883,7 @@ mla_status mla_decode_noalloc(const mla_dims *d, const void *q, const mla_cache 
   if (static_cast<int64_t>(B) * n_q > NOALLOC_MAX_ROWS)
     return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc serves at most %d token rows (B * n_q), got %lld",
                 NOALLOC_MAX_ROWS, static_cast<long long>(B) * n_q);
-  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_DECODE, B, n_q, 0, 0);
   if (need > NOALLOC_BYTES)
     return fail(MLA_ERR_UNSUPPORTED, "mla_decode_noalloc: this call needs %zu scratch bytes, %zu are reserved", need,
                 NOALLOC_BYTES);
@@ -867,7 +900,7 @@ mla_status mla_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, 
   if (!o_lat || !W_UV || !o) return fail(MLA_ERR_INVALID_ARG, "out_proj: NULL tensor argument");
   if (!aligned16(o_lat) || !aligned16(W_UV) || !aligned16(o))
     return fail(MLA_ERR_INVALID_ARG, "out_proj: tensors must be 16-byte aligned");
-  const size_t need = mla_workspace_size(d, MLA_OP_OUT_PROJ, T, 1, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_OUT_PROJ, T, 1, 0, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "out_proj needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_geometry(d)) return tc_out_proj(d, o_lat, W_UV, T, o, ws, st);
@@ -884,7 +917,7 @@ mla_status mla_o_proj(const mla_dims *d, const void *o, const void *W_O, int32_t
   if (!aligned16(o) || !aligned16(W_O) || !aligned16(y))
     return fail(MLA_ERR_INVALID_ARG, "o_proj: tensors must be 16-byte aligned");
   if (d->d % 2 != 0) return fail(MLA_ERR_UNSUPPORTED, "o_proj: d must be even");
-  const size_t need = mla_workspace_size(d, MLA_OP_O_PROJ, T, 1, 0);
+  const size_t need = mla_workspace_size(d, MLA_OP_O_PROJ, T, 1, 0, 0);
   if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "o_proj needs %zu workspace bytes", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_geometry(d)) return tc_o_proj(d, o, W_O, T, y, ws, st);

@@ -47,7 +47,7 @@ _lib.mla_decode.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_i
 _lib.mla_out_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
 _lib.mla_o_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
 _lib.mla_decode_noalloc.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P, _P]
-_lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64]
+_lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_int32]
 _lib.mla_workspace_size.restype = C.c_size_t
 _lib.mla_get_device_error.argtypes = [_P]
 _lib.mla_status_string.argtypes = [C.c_int]
@@ -109,12 +109,18 @@ class Cache:
                                   block_table.shape[1], block_table.shape[0], 0, data.shape[0])
 
 
-def workspace_size(p: Dims, op: int, rows: int, n_q: int = 1, max_seq_len: int = 0) -> int:
-    return int(_lib.mla_workspace_size(C.byref(p), op, rows, n_q, max_seq_len))
+def workspace_size(p: Dims, op: int, rows: int, n_q: int = 1, max_seq_len: int = 0, num_splits: int = 0) -> int:
+    return int(_lib.mla_workspace_size(C.byref(p), op, rows, n_q, max_seq_len, num_splits))
 
 
-def _ws(p, op, rows, n_q, ws):
-    need = workspace_size(p, op, rows, n_q)
+def cache_capacity(cache: "Cache") -> int:
+    """Longest sequence the cache can hold (the bound mla_decode sizes forced splits by)."""
+    d = cache.desc
+    return d.max_blocks_per_seq * d.block_size if d.paged else d.max_len
+
+
+def _ws(p, op, rows, n_q, ws, max_seq_len=0, num_splits=0):
+    need = workspace_size(p, op, rows, n_q, max_seq_len, num_splits)
     if ws is None and need > 0:
         ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     return ws, need if ws is None else ws.numel()
@@ -143,7 +149,7 @@ def mla_absorb_q(p: Dims, h, W_DQ, W_UQ, W_QR, W_UK, positions, q, ws=None, stre
 def mla_decode(p: Dims, q, cache: Cache, seq_lens, n_q, o_lat, lse=None, num_splits=0, ws=None,
                stream=None):
     B = seq_lens.shape[0]
-    ws, nbytes = _ws(p, OP_DECODE, B, n_q, ws)
+    ws, nbytes = _ws(p, OP_DECODE, B, n_q, ws, cache_capacity(cache), num_splits)
     _check(_lib.mla_decode(C.byref(p), _ptr(q), C.byref(cache.desc), _ptr(seq_lens), B, n_q,
                            _ptr(o_lat), _ptr(lse), num_splits, _ptr(ws), nbytes, _stream(stream)),
            "mla_decode")

@@ -135,6 +135,8 @@ int64_t orc_slot(const orc_cache *c, int32_t b, int64_t pos) {
 void orc_append(const orc_dims *p, const double *h, const double *W_DKV, const double *W_KR,
                 const int32_t *positions, int T, double *rows) {
   const int D = p->d_c + p->d_r;
+  /* token rows are independent: one row per OpenMP iteration */
+#pragma omp parallel for schedule(dynamic, 1)
   for (int t = 0; t < T; ++t) {
     const double *ht = h + (int64_t)t * p->d;
     double *out = rows + (int64_t)t * D;
@@ -152,8 +154,13 @@ void orc_absorb_q(const orc_dims *p, const double *h, const double *W_DQ, const 
                   const double *W_QR, const double *W_UK, const int32_t *positions, int T,
                   double *q_out, double *q_C_out) {
   const int D = p->d_c + p->d_r;
+  /* token rows are independent: one row per OpenMP iteration, each thread
+   * with its own c_Q and q_C scratch */
+#pragma omp parallel
+  {
   double *cq = (double *)malloc(sizeof(double) * p->d_cq);
   double *qc = (double *)malloc(sizeof(double) * p->d_h);
+#pragma omp for schedule(dynamic, 1)
   for (int t = 0; t < T; ++t) {
     orc_matvec(W_DQ, p->d_cq, p->d, h + (int64_t)t * p->d, cq);
     for (int hh = 0; hh < p->n_h; ++hh) {
@@ -173,6 +180,7 @@ void orc_absorb_q(const orc_dims *p, const double *h, const double *W_DQ, const 
   }
   free(cq);
   free(qc);
+  }
 }
 
 /* Order B for one (query row, head) over cached positions [start, end) of
@@ -273,6 +281,7 @@ void orc_combine(int S, int d_c, const double *o_parts, const double *lse_parts,
 
 /* Step 2 + step 5 readout (eq. 11): o[t][h*d_h + i] = sum_j W_UV[h*d_h+i][j] o_lat[t][h][j]. */
 void orc_out_proj(const orc_dims *p, const double *o_lat, const double *W_UV, int T, double *o) {
+#pragma omp parallel for schedule(dynamic, 1)
   for (int t = 0; t < T; ++t)
     for (int hh = 0; hh < p->n_h; ++hh)
       orc_matvec(W_UV + (int64_t)hh * p->d_h * p->d_c, p->d_h, p->d_c,
@@ -285,6 +294,7 @@ void orc_out_proj(const orc_dims *p, const double *o_lat, const double *W_UV, in
  * width by W_O (d x n_h*d_h): y_t = W x_t for every token row t. The same
  * routine applies the absorbed matrix of orc_absorb_wo to o_lat. */
 void orc_o_proj(const double *W, int rows, int cols, const double *x, int T, double *y) {
+#pragma omp parallel for schedule(dynamic, 1)
   for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)t * cols, y + (int64_t)t * rows);
 }
 

@@ -24,7 +24,7 @@ def mla():
     return m
 
 
-def _run(mla, orc, w, seed, seq_lens, n_q=1, check_lse=True, pairs=None):
+def _run(mla, orc, w, seed, seq_lens, n_q=1, check_lse=True, pairs=None, num_splits=0):
     import torch
     from tests.gpu_util import assert_close, dev, dims_of, orc_dims_of, host
     w = synth.shrink(w, n_q=n_q)
@@ -40,7 +40,7 @@ def _run(mla, orc, w, seed, seq_lens, n_q=1, check_lse=True, pairs=None):
     o_lat = torch.full((T, w.n_h, w.d_c), float("nan"), device="cuda",
                        dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
     lse = torch.full((T, w.n_h), float("nan"), device="cuda", dtype=torch.float32)
-    mla.mla_decode(p, q, cache, sl, n_q, o_lat, lse)
+    mla.mla_decode(p, q, cache, sl, n_q, o_lat, lse, num_splits=num_splits)
     assert mla.mla_get_device_error() == mla.MLA_OK
     oc = orc.Cache(x.cache, x.block_table)
     po = orc_dims_of(w, orc)
@@ -90,6 +90,28 @@ def test_decode_tc_many_short_sequences(mla, orc):
     # more rows than clusters: several rows per cluster, most finished in place
     rng = np.random.default_rng(14)
     _run(mla, orc, V2, 14, list(rng.integers(1, 300, size=300)))
+
+
+# Split-KV independence: forced split counts S (each token row cut into
+# min(S, its tiles) pieces, merged by the log-sum-exp combine) and the
+# automatic plan (S = 0) all match the oracle.
+SPLIT_LENS = [3000, 1, 700, 5000, 257, 64, 1800]
+
+
+@pytest.mark.parametrize("splits", [1, 2, 7, 0])
+def test_decode_tc_split_independence(mla, orc, splits):
+    _run(mla, orc, V2, 23, SPLIT_LENS, num_splits=splits)
+
+
+@pytest.mark.parametrize("splits", [3, 74])
+def test_decode_tc_forced_splits_two_queries(mla, orc, splits):
+    # 74 pieces ask for more than the tiles of every row here: one tile per piece
+    _run(mla, orc, V2, 24, [2, 513, 4000, 9000], n_q=2, num_splits=splits)
+
+
+def test_decode_tc_forced_splits_long_rows(mla, orc):
+    # long rows cut into more pieces than there are clusters
+    _run(mla, orc, V2, 25, [30000, 20011], num_splits=200)
 
 
 def test_decode_tc_two_queries_causal(mla, orc):

@@ -1,7 +1,8 @@
 """Output projection y = W_O o (MLA walk-through, section 1 step 5) through
 the C ABI against the fp64 oracle, element by element: DeepSeek-V2 dims on
 the tensor cores (split-K GEMM + finalize; several tiles and a ragged token
-tail) and the fp32 tiny dims on the CUDA cores."""
+tail, up to 200 token rows) and the tiny dims on the CUDA cores in fp32 and
+bf16 storage."""
 import numpy as np
 import pytest
 
@@ -19,14 +20,18 @@ def mla():
     return m
 
 
+TINY_BF16 = synth.shrink(synth.WORKLOADS["tiny_fp32"], dtype="bf16")
+
+
 @pytest.mark.parametrize("name,T", [("v2_b64_paged", 1), ("v2_b64_paged", 37), ("v2_b64_paged", 64),
-                                    ("tiny_fp32", 5)])
+                                    ("v2_b64_paged", 200), ("tiny_fp32", 5), ("tiny_bf16", 7)])
 def test_o_proj_matches_oracle(mla, name, T):
     import torch
     import oracle as orc
     from tests.gpu_util import assert_close, dev, dims_of, host
-    w = synth.WORKLOADS[name]
+    w = TINY_BF16 if name == "tiny_bf16" else synth.WORKLOADS[name]
     p = dims_of(w, mla)
+    assert mla.uses_tensor_cores(p, mla.OP_O_PROJ) == (name == "v2_b64_paged")
     HD = w.n_h * w.d_h
     rng = np.random.default_rng(4242 + T)
     W_O = rng.standard_normal((w.d, HD), dtype=np.float32) / np.float32(np.sqrt(HD))

@@ -27,6 +27,8 @@ CASES = {
     "v2_paged_T5": synth.shrink(synth.WORKLOADS["v2_b64_paged"], B=5, L_lo=1, L_hi=300),
     "v3_paged_T6_nq2": synth.shrink(synth.WORKLOADS["v3_b128_nq2"], B=3, L_lo=2, L_hi=200),
     "v2_contig_T3": synth.shrink(synth.WORKLOADS["v2_b16_4k"], B=3, L=77),
+    # 256 token rows: the absorb runs as [W_UQ; W_QR] then the per-head W_UK^T GEMM through the workspace
+    "v3_paged_T256_nq2": synth.shrink(synth.WORKLOADS["v3_b128_nq2"], L_lo=2, L_hi=150, median=60.0),
     "tiny_fp32": synth.WORKLOADS["tiny_fp32"],
     "small_bf16": synth.Workload("small_bf16", 9, d=96, n_h=3, d_h=16, d_c=32, d_cq=48, d_r=8, B=4,
                                  n_q=1, lens="uniform", L_lo=1, L_hi=40, paged=True, block_size=16),
@@ -137,8 +139,8 @@ def test_host_validation_rejects_bad_arguments(mla):
         mla.mla_decode(p, q[:, :, 1:], cache, sl, 1, o)  # misaligned base (2-byte offset)
     assert e.value.status == mla.MLA_ERR_INVALID_ARG
     with pytest.raises(mla.MlaError) as e:
-        mla.mla_decode(p, q, cache, sl, 1, o, num_splits=3)
-    assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+        mla.mla_decode(p, q, cache, sl, 1, o, num_splits=-1)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode(p, q, cache, sl, 1, o, ws=torch.zeros(16, dtype=torch.uint8, device="cuda"))
     assert e.value.status == mla.MLA_ERR_WORKSPACE

@@ -86,7 +86,7 @@ def test_append_arguments(m):
     assert append(m, d, cache=paged_cache(m, data=MIS)) == m.MLA_ERR_INVALID_ARG
     assert append(m, d, cache=m.CacheDesc(A, 0, 0, None, 0, 4, 0, 0)) == m.MLA_ERR_INVALID_ARG
     assert "max_len" in last_msg(m)
-    need = m._lib.mla_workspace_size(C.byref(d), m.OP_APPEND, 64, 1, 0)
+    need = m._lib.mla_workspace_size(C.byref(d), m.OP_APPEND, 64, 1, 0, 0)
     assert need > 0
     assert append(m, d, ws_bytes=need - 1) == m.MLA_ERR_WORKSPACE and str(need) in last_msg(m)
     assert append(m, d, ws=None, ws_bytes=need) == m.MLA_ERR_WORKSPACE
@@ -97,15 +97,15 @@ def test_absorb_and_out_proj_arguments(m):
     ab = m._lib.mla_absorb_q
     assert ab(C.byref(d), A, A, A, A, A, A, 64, MIS, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
     assert ab(C.byref(d), A, A, A, A, None, A, 64, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
-    need = m._lib.mla_workspace_size(C.byref(d), m.OP_ABSORB, 64, 1, 0)
+    need = m._lib.mla_workspace_size(C.byref(d), m.OP_ABSORB, 64, 1, 0, 0)
     assert need > 0
     assert ab(C.byref(d), A, A, A, A, A, A, 64, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
     op = m._lib.mla_out_proj
     assert op(C.byref(d), A, A, 0, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
     assert op(C.byref(d), MIS, A, 64, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
     # the tensor-core out-projection needs no workspace (one CTA per head, no split-K)
-    assert m._lib.mla_workspace_size(C.byref(d), m.OP_OUT_PROJ, 64, 1, 0) == 0
-    need = m._lib.mla_workspace_size(C.byref(v2(m, dtype="fp32")), m.OP_OUT_PROJ, 64, 1, 0)
+    assert m._lib.mla_workspace_size(C.byref(d), m.OP_OUT_PROJ, 64, 1, 0, 0) == 0
+    need = m._lib.mla_workspace_size(C.byref(v2(m, dtype="fp32")), m.OP_OUT_PROJ, 64, 1, 0, 0)
     assert need > 0  # the CUDA-core path keeps fp32 intermediate rows
     assert op(C.byref(v2(m, dtype="fp32")), A, A, 64, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
 
@@ -116,7 +116,7 @@ def test_o_proj_arguments(m):
     assert op(C.byref(d), A, A, 0, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
     assert op(C.byref(d), A, None, 64, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
     assert op(C.byref(d), A, A, 64, MIS, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG and "aligned" in last_msg(m)
-    need = m._lib.mla_workspace_size(C.byref(d), m.OP_O_PROJ, 64, 1, 0)
+    need = m._lib.mla_workspace_size(C.byref(d), m.OP_O_PROJ, 64, 1, 0, 0)
     assert 0 < need < 1 << 30  # split-K fp32 partials of the 5120 x 64 output
     assert op(C.byref(d), A, A, 64, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
 
@@ -129,11 +129,18 @@ def test_decode_arguments(m):
     assert decode(m, d, o_lat=MIS) == m.MLA_ERR_INVALID_ARG and "aligned" in last_msg(m)
     assert decode(m, d, B=65) == m.MLA_ERR_INVALID_ARG and "num_seqs" in last_msg(m)
     assert decode(m, d, num_splits=-1) == m.MLA_ERR_INVALID_ARG
-    need = m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, 0)
+    need = m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, 0, 0)
     assert 0 < need < 1 << 30
     assert decode(m, d, ws_bytes=need - 1) == m.MLA_ERR_WORKSPACE
-    # the tensor-core decode plans its own split of the work
-    assert decode(m, d, num_splits=4) == m.MLA_ERR_UNSUPPORTED and "num_splits = 0" in last_msg(m)
+    # forced splits: partials for min(S, tiles of the longest row the cache holds) pieces of every row;
+    # the paged cache here holds 128 blocks of 64 = 8192 tokens = 32 tiles per row
+    cap = 128 * 64
+    need4 = m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, cap, 4)
+    need64 = m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, cap, 64)
+    assert need64 > need4 >= need
+    assert need64 == m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, cap, 32)  # capped at 32 tiles
+    assert m._lib.mla_workspace_size(C.byref(d), m.OP_DECODE, 64, 1, 0, 64) > need64      # unknown length: 64 per row
+    assert decode(m, d, num_splits=64, ws_bytes=need64 - 1) == m.MLA_ERR_WORKSPACE
 
 
 def test_noalloc_decode_limit(m):
@@ -145,14 +152,14 @@ def test_noalloc_decode_limit(m):
 
 def test_workspace_sizes(m):
     d = v2(m)
-    ws = lambda op, rows, n_q=1: m._lib.mla_workspace_size(C.byref(d), op, rows, n_q, 0)
+    ws = lambda op, rows, n_q=1: m._lib.mla_workspace_size(C.byref(d), op, rows, n_q, 0, 0)
     # decode: a plan plus fp32 partials of 128 x 512 (and 128 lse) per slot,
     # slots = token rows + clusters; more rows never need less
     assert ws(m.OP_DECODE, 64) > 64 * 128 * 512 * 4
     assert ws(m.OP_DECODE, 128) > ws(m.OP_DECODE, 64)
     assert ws(m.OP_DECODE, 64, 2) > ws(m.OP_DECODE, 64, 1)
     assert ws(m.OP_DECODE, 0) == 0 and ws(m.OP_APPEND, -1) == 0
-    assert m._lib.mla_workspace_size(None, m.OP_DECODE, 64, 1, 0) == 0
+    assert m._lib.mla_workspace_size(None, m.OP_DECODE, 64, 1, 0, 0) == 0
     assert ws(7, 64) == 0  # unknown op
 
 

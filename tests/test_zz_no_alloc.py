@@ -38,22 +38,50 @@ def _outputs(w):
             torch.full((T, w.n_h), float("nan"), device="cuda", dtype=torch.float32))
 
 
-@pytest.mark.parametrize("seq_lens,n_q", [
+CASES = [
     (list(np.random.default_rng(42).integers(1, 3000, size=64)), 1),  # the 64-row limit, rows cut between clusters
     ([2, 65, 700, 4099, 257, 3], 2),
-])
-def test_noalloc_matches_workspace_decode_twice(mla, seq_lens, n_q):
+]
+
+
+@pytest.mark.parametrize("overlap", [False, True])
+@pytest.mark.parametrize("seq_lens,n_q", CASES)
+def test_noalloc_matches_workspace_decode_twice(mla, seq_lens, n_q, overlap):
+    """Two no-alloc calls enqueued back to back on one stream (with launch
+    overlap on, the second call's decode may start while the first call's
+    combine still reads the shared scratch), then one synchronisation."""
     from tests.gpu_util import assert_close, host
     w, p, q, cache, sl = _inputs(mla, seq_lens, n_q)
     ref_o, ref_l = _outputs(w)
     mla.mla_decode(p, q, cache, sl, n_q, ref_o, ref_l)
     assert mla.mla_get_device_error() == mla.MLA_OK
-    for _ in range(2):
-        o, l = _outputs(w)
-        mla.mla_decode_noalloc(p, q, cache, sl, n_q, o, l)
+    was = mla.get_launch_overlap()
+    mla.set_launch_overlap(overlap)
+    try:
+        outs = [_outputs(w) for _ in range(2)]
+        for o, l in outs:
+            mla.mla_decode_noalloc(p, q, cache, sl, n_q, o, l)
         assert mla.mla_get_device_error() == mla.MLA_OK
+    finally:
+        mla.set_launch_overlap(was)
+    for o, l in outs:
         assert_close(host(o), host(ref_o), "o_lat (no-alloc vs workspace)")
         assert_close(host(l), host(ref_l), "lse (no-alloc vs workspace)")
+
+
+def test_noalloc_matches_oracle(mla, orc):
+    """The 64-row case against the fp64 oracle directly."""
+    from tests.gpu_util import assert_close, host, orc_dims_of
+    seq_lens, n_q = CASES[0]
+    w0 = synth.shrink(synth.WORKLOADS["v2_b64_paged"], n_q=n_q)
+    x = synth.generate_decode(w0, 41, seq_lens=seq_lens)
+    w, p, q, cache, sl = _inputs(mla, seq_lens, n_q)
+    o, l = _outputs(w)
+    mla.mla_decode_noalloc(p, q, cache, sl, n_q, o, l)
+    assert mla.mla_get_device_error() == mla.MLA_OK
+    ref_o, ref_l = orc.decode(orc_dims_of(w, orc), x.q, orc.Cache(x.cache, x.block_table), x.seq_lens, n_q)
+    assert_close(host(o), ref_o, "o_lat (no-alloc vs oracle)")
+    assert_close(host(l), ref_l, "lse (no-alloc vs oracle)")
 
 
 def test_noalloc_rejects_more_rows_than_its_scratch(mla):
