@@ -53,6 +53,7 @@ def bind(L):
     L.orc_decode_order_a.restype = C.c_int
     L.orc_o_proj.argtypes = [_P, C.c_int, C.c_int, _P, C.c_int, _P]
     L.orc_absorb_wo.argtypes = [C.POINTER(OrcDims), _P, _P, _P]
+    L.orc_absorb_merge.argtypes = [C.POINTER(OrcDims), _P, _P, _P]
     L.orc_set_threads.argtypes = [C.c_int]
     L.orc_max_threads.restype = C.c_int
     return L
@@ -210,6 +211,14 @@ def absorb_wo(p: OrcDims, W_O, W_UV):
     return W_OV
 
 
+def absorb_merge(p: OrcDims, W_UQ, W_UK):
+    """W_UQK (n_h*d_c x d_cq): the merged absorption matrix W_UK_h^T W_UQ_h per head."""
+    W_UQ, W_UK = _f64(W_UQ), _f64(W_UK)
+    W_UQK = np.empty((p.n_h * p.d_c, p.d_cq))
+    lib().orc_absorb_merge(C.byref(p), _ptr(W_UQ), _ptr(W_UK), _ptr(W_UQK))
+    return W_UQK
+
+
 def decode_order_a(p: OrcDims, q_C, q_R, W_UK, W_UV, cache: Cache, seq_lens, n_q, pairs=None):
     """Order A (decompress per head, then ordinary attention). Returns o per
     head: [T][n_h][d_h] or [n_pairs][d_h]."""
@@ -256,5 +265,6 @@ def step(p: OrcDims, w, h, positions, seq_idx, cache_rows_before: Cache, seq_len
 
 
 __all__ = ["dims", "Cache", "rope", "append_rows", "absorb_q", "decode", "attend_range",
-           "combine", "out_proj", "decode_order_a", "step", "set_threads", "max_threads"]
+           "combine", "out_proj", "decode_order_a", "step", "set_threads", "max_threads", "o_proj",
+           "absorb_wo", "absorb_merge"]
 

@@ -305,6 +305,8 @@ void orc_o_proj(const double *W, int rows, int cols, const double *x, int T, dou
  * a d x n_h*d_c matrix. W_O is d x n_h*d_h, W_UV is n_h*d_h x d_c. */
 void orc_absorb_wo(const orc_dims *p, const double *W_O, const double *W_UV, double *W_OV) {
   const int64_t ko = (int64_t)p->n_h * p->d_h, kv = (int64_t)p->n_h * p->d_c;
+  /* rows r are independent: one row per OpenMP iteration */
+#pragma omp parallel for schedule(dynamic, 1)
   for (int r = 0; r < p->d; ++r)
     for (int hh = 0; hh < p->n_h; ++hh)
       for (int j = 0; j < p->d_c; ++j) {
@@ -312,6 +314,24 @@ void orc_absorb_wo(const orc_dims *p, const double *W_O, const double *W_UV, dou
         for (int i = 0; i < p->d_h; ++i)
           acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[((int64_t)hh * p->d_h + i) * p->d_c + j];
         W_OV[r * kv + (int64_t)hh * p->d_c + j] = acc;
+      }
+}
+
+/* Merged absorption matrix (walk-through, section 3 order B: the product of
+ * the two matrices absorbed on the query side can be formed offline):
+ * W_UQK_h = W_UK_h^T W_UQ_h, so that q_lat,h = W_UQK_h c_Q in one product,
+ *   W_UQK[h*d_c + j][c] = sum_i W_UK[h*d_h + i][j] W_UQ[h*d_h + i][c].
+ * W_UQ is n_h*d_h x d_cq, W_UK is n_h*d_h x d_c, W_UQK is n_h*d_c x d_cq. */
+void orc_absorb_merge(const orc_dims *p, const double *W_UQ, const double *W_UK, double *W_UQK) {
+  /* heads are independent: one head per OpenMP iteration */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int hh = 0; hh < p->n_h; ++hh)
+    for (int j = 0; j < p->d_c; ++j)
+      for (int c = 0; c < p->d_cq; ++c) {
+        double acc = 0.0;
+        for (int i = 0; i < p->d_h; ++i)
+          acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ[((int64_t)hh * p->d_h + i) * p->d_cq + c];
+        W_UQK[((int64_t)hh * p->d_c + j) * p->d_cq + c] = acc;
       }
 }
 

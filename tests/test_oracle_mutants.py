@@ -42,6 +42,12 @@ MUTANTS = [
     ("W_O absorption reads W_UV transposed",
      "acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[((int64_t)hh * p->d_h + i) * p->d_c + j];",
      "acc += W_O[r * ko + (int64_t)hh * p->d_h + i] * W_UV[(int64_t)hh * p->d_h * p->d_c + (int64_t)j * p->d_h + i];"),
+    ("merged absorption reads W_UQ transposed",
+     "acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ[((int64_t)hh * p->d_h + i) * p->d_cq + c];",
+     "acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ[(int64_t)hh * p->d_h * p->d_cq + (int64_t)c * p->d_h + i];"),
+    ("merged absorption drops the last head row",
+     "        for (int i = 0; i < p->d_h; ++i)\n          acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ",
+     "        for (int i = 0; i < p->d_h - 1; ++i)\n          acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ"),
     ("output projection skips a token row",
      "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)t * cols, y + (int64_t)t * rows);",
      "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)(t > 0 ? t - 1 : 0) * cols, y + (int64_t)t * rows);"),

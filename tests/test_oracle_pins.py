@@ -306,6 +306,26 @@ def test_absorbed_w_o_matches_library_and_the_two_stage_readout(orc):
     assert np.allclose(one_stage, two_stage, rtol=1e-12, atol=1e-13)
 
 
+def test_merged_absorption_matches_the_two_stage_query(orc):
+    # the merged matrix W_UK_h^T W_UQ_h (walk-through section 3, order B): applied to c_Q it
+    # gives the oracle's own two-stage q_lat (W_UQ, then W_UK^T), which the library-chain and
+    # order-A pins fix independently; and it is the per-head product of the library
+    rng = np.random.default_rng(14)
+    w, _, dm = _rand_problem(rng)
+    p = orc.dims(**dm)
+    n_h, d_h, d_c, d_cq = dm["n_h"], dm["d_h"], dm["d_c"], dm["d_cq"]
+    W_UQK = orc.absorb_merge(p, w["W_UQ"], w["W_UK"])
+    assert W_UQK.shape == (n_h * d_c, d_cq)
+    T = 3
+    h = rng.standard_normal((T, dm["d"]))
+    q = orc.absorb_q(p, h, w["W_DQ"], w["W_UQ"], w["W_QR"], w["W_UK"], np.arange(T, dtype=np.int32))
+    cq = h @ w["W_DQ"].T
+    for hh in range(n_h):
+        assert np.allclose(cq @ W_UQK[hh * d_c:(hh + 1) * d_c].T, q[:, hh, :d_c], rtol=1e-11, atol=1e-12)
+    ref = np.einsum("hij,hic->hjc", w["W_UK"].reshape(n_h, d_h, d_c), w["W_UQ"].reshape(n_h, d_h, d_cq))
+    assert np.allclose(W_UQK, ref.reshape(n_h * d_c, d_cq), rtol=1e-13, atol=1e-14)
+
+
 def test_bf16_cache_read_is_exact(orc):
     # the oracle reads bf16 storage as the exact real value of those bits
     vals = np.array([1.0, -2.5, 3.140625, 1e-3, 65280.0], np.float32)
