@@ -74,7 +74,19 @@ def parse():
                     help="mla_decode num_splits: 0 = automatic plan, S > 0 = each token row in min(S, its tiles) pieces")
     ap.add_argument("--with-o-proj", action="store_true",
                     help="add the output projection y = W_O o (mla_o_proj) to every step and time it on its own")
-    return ap.parse_args()
+    ap.add_argument("--o-proj-absorbed", action="store_true",
+                    help="with --with-o-proj: y = W_OV o_lat (mla_o_proj_latent, W_UV absorbed into W_O) in place of "
+                         "the W_UV readout and W_O")
+    ap.add_argument("--fused-front-end", action="store_true",
+                    help="append and absorb in one call (mla_front_end: h read once) instead of two calls on two streams")
+    ap.add_argument("--merged-absorb", action="store_true",
+                    help="absorb with the merged matrix W_UK_h^T W_UQ_h (mla_absorb_q_merged)")
+    a = ap.parse_args()
+    if a.o_proj_absorbed and not a.with_o_proj:
+        ap.error("--o-proj-absorbed needs --with-o-proj")
+    if a.merged_absorb and a.fused_front_end:
+        ap.error("--merged-absorb and --fused-front-end are exclusive")
+    return a
 
 
 L2_BYTES = 126 * 1024 * 1024
@@ -221,20 +233,30 @@ def run_ours(args, rank, world, local_rank):
         rng = np.random.Generator(np.random.PCG64(2000 + w.index))
         W_O = rng.standard_normal((w.d, HD), dtype=np.float32) * np.float32(1.0 / math.sqrt(HD))
         W["W_O"] = torch.from_numpy(synth.bf16_bits(W_O).view(np.int16)).view(torch.bfloat16).to(dev)
-        y = torch.empty((T, w.d), device=dev, dtype=torch.bfloat16)
+        if args.o_proj_absorbed:  # offline: W_OV = W_O blockdiag(W_UV_h), before any timing
+            W["W_OV"] = torch.empty((w.d, w.n_h * w.d_c), device=dev, dtype=torch.bfloat16)
+            mla.mla_absorb_wo(p, W["W_O"], W["W_UV"], W["W_OV"])
+    if args.merged_absorb:  # offline: W_UQK_h = W_UK_h^T W_UQ_h, before any timing
+        W["W_UQK"] = torch.empty((w.n_h * w.d_c, w.d_cq), device=dev, dtype=torch.bfloat16)
+        mla.mla_absorb_merge(p, W["W_UQ"], W["W_UK"], W["W_UQK"])
+    torch.cuda.synchronize()
     # two sets of the step's input and output buffers, so that the end-to-end
     # loop can copy the next step's inputs in while this step computes
     h_host = torch.from_numpy(x.h_bits.view(np.int16)).view(torch.bfloat16)
     bufs = [{"h": h_host.to(dev), "pos": torch.from_numpy(x.positions).to(dev),
              "sidx": torch.from_numpy(x.seq_idx).to(dev), "sl": torch.from_numpy(x.seq_lens).to(dev),
-             "o": torch.empty((T, w.n_h * w.d_h), device=dev, dtype=torch.bfloat16)} for _ in range(2)]
-    o = bufs[0]["o"]
+             "o": torch.empty((T, w.n_h * w.d_h), device=dev, dtype=torch.bfloat16),
+             "y": torch.empty((T, w.d), device=dev, dtype=torch.bfloat16) if args.with_o_proj else None}
+            for _ in range(2)]
+    out_key = "y" if args.with_o_proj else "o"  # what a step hands back to the host
+    o = bufs[0][out_key]
     q = torch.empty((T, w.n_h, w.D), device=dev, dtype=torch.bfloat16)
     o_lat = torch.empty((T, w.n_h, w.d_c), device=dev, dtype=torch.bfloat16)
     lse = torch.empty((T, w.n_h), device=dev, dtype=torch.float32)
     ws = {op: torch.empty(max(1, mla.workspace_size(p, op, w.B if op == mla.OP_DECODE else T, w.n_q)),
                           dtype=torch.uint8, device=dev)
-          for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ, mla.OP_O_PROJ)}
+          for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ, mla.OP_O_PROJ,
+                     mla.OP_O_PROJ_LATENT, mla.OP_ABSORB_MERGED, mla.OP_FRONT_END)}
     ws[mla.OP_DECODE] = torch.empty(max(1, mla.workspace_size(p, mla.OP_DECODE, w.B, w.n_q, mla.cache_capacity(caches[0]),
                                                               args.num_splits)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)  # graph capture needs a non-default stream
@@ -253,25 +275,37 @@ def run_ours(args, rank, world, local_rank):
     def step(i=None, b=0, c=None):
         x_ = bufs[b]
         cache = caches[(i if c is None else c) % n_copies if (i is not None or c is not None) else 0]
-        ev_fork.record(stream)
-        side.wait_event(ev_fork)
-        mla.mla_cache_append(p, x_["h"], W["W_DKV"], W["W_KR"], x_["sidx"], x_["pos"], cache,
-                             ws=ws[mla.OP_APPEND], stream=side)
-        ev_join.record(side)
-        mla.mla_absorb_q(p, x_["h"], W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], x_["pos"], q,
-                         ws=ws[mla.OP_ABSORB], stream=stream)
-        stream.wait_event(ev_join)
+        if args.fused_front_end:
+            mla.mla_front_end(p, x_["h"], W["W_DKV"], W["W_KR"], W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"],
+                              x_["sidx"], x_["pos"], cache, q, ws=ws[mla.OP_FRONT_END], stream=stream)
+        else:
+            ev_fork.record(stream)
+            side.wait_event(ev_fork)
+            mla.mla_cache_append(p, x_["h"], W["W_DKV"], W["W_KR"], x_["sidx"], x_["pos"], cache,
+                                 ws=ws[mla.OP_APPEND], stream=side)
+            ev_join.record(side)
+            if args.merged_absorb:
+                mla.mla_absorb_q_merged(p, x_["h"], W["W_DQ"], W["W_UQK"], W["W_QR"], x_["pos"], q,
+                                        ws=ws[mla.OP_ABSORB_MERGED], stream=stream)
+            else:
+                mla.mla_absorb_q(p, x_["h"], W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"], x_["pos"], q,
+                                 ws=ws[mla.OP_ABSORB], stream=stream)
+            stream.wait_event(ev_join)
         if i is not None:
             ev_dec[i][0].record(stream)
         mla.mla_decode(p, q, cache, x_["sl"], w.n_q, o_lat, lse, num_splits=args.num_splits, ws=ws[mla.OP_DECODE],
                        stream=stream)
         if i is not None:
             ev_dec[i][1].record(stream)
-        mla.mla_out_proj(p, o_lat, W["W_UV"], x_["o"], ws=ws[mla.OP_OUT_PROJ], stream=stream)
+        if not args.o_proj_absorbed:
+            mla.mla_out_proj(p, o_lat, W["W_UV"], x_["o"], ws=ws[mla.OP_OUT_PROJ], stream=stream)
         if args.with_o_proj:
             if i is not None:
                 ev_op[i][0].record(stream)
-            mla.mla_o_proj(p, x_["o"], W["W_O"], y, ws=ws[mla.OP_O_PROJ], stream=stream)
+            if args.o_proj_absorbed:
+                mla.mla_o_proj_latent(p, o_lat, W["W_OV"], x_["y"], ws=ws[mla.OP_O_PROJ_LATENT], stream=stream)
+            else:
+                mla.mla_o_proj(p, x_["o"], W["W_O"], x_["y"], ws=ws[mla.OP_O_PROJ], stream=stream)
             if i is not None:
                 ev_op[i][1].record(stream)
 
@@ -380,7 +414,7 @@ def run_ours(args, rank, world, local_rank):
             ev_done[b].record(stream)
         with torch.cuda.stream(d2h_stream):
             d2h_stream.wait_event(ev_done[b])
-            o_host[b].copy_(bufs[b]["o"], non_blocking=True)
+            o_host[b].copy_(bufs[b][out_key], non_blocking=True)
             ev_out[b].record(d2h_stream)
     stream.wait_stream(h2d_stream)
     stream.wait_stream(d2h_stream)
@@ -500,6 +534,19 @@ def run_reference(args, rank, world):
     print(json.dumps(line))
 
 
+def step_text(args):
+    if args is None:
+        return "append + absorb + decode + W_UV readout"
+    front = ("fused front end (append + absorb, h read once)" if args.fused_front_end else
+             "append + " + ("merged-matrix absorb" if args.merged_absorb else "absorb"))
+    tail = " + decode"
+    if args.with_o_proj:
+        tail += " + W_OV o_lat (W_UV absorbed into W_O)" if args.o_proj_absorbed else " + W_UV readout + W_O projection"
+    else:
+        tail += " + W_UV readout"
+    return front + tail
+
+
 def config_of(w, n, x, n_copies=None, args=None):
     L = x.seq_lens
     cache_bytes = int(x.cache.nbytes)
@@ -515,12 +562,17 @@ def config_of(w, n, x, n_copies=None, args=None):
             "dims": {"d": w.d, "n_h": w.n_h, "d_h": w.d_h, "d_c": w.d_c, "d_cq": w.d_cq, "d_r": w.d_r},
             "parallelism": f"replicas{n}", "seed": 1000 + w.index, "l2": l2,
             "num_splits": 0 if args is None else args.num_splits,
-            "step": "append + absorb + decode + W_UV readout" + (" + W_O projection" if args is not None and
-                                                                 args.with_o_proj else "")}
+            "step": step_text(args)}
 
 
-def HD_of(w):
-    return w.n_h * w.d_h
+def o_proj_line(w, op_ms, peaks, absorbed):
+    """Timing of the output projection against its weight-streaming roofline:
+    W_O (d x n_h d_h) or, absorbed, W_OV (d x n_h d_c), bf16."""
+    k = w.n_h * (w.d_c if absorbed else w.d_h)
+    wb = w.d * k * 2
+    return {"kernel": "mla_o_proj_latent (W_OV o_lat)" if absorbed else "mla_o_proj (W_O o)", "us": op_ms * 1e3,
+            "weight_bytes": wb, "gbs": wb / (op_ms * 1e-3) / 1e9,
+            "frac": (wb / (peaks["hbm_gbs"] * 1e9)) / (op_ms * 1e-3), "peak_gbs": peaks["hbm_gbs"]}
 
 
 def main():
@@ -584,10 +636,7 @@ def main():
         "e2e": {"value": r["e2e_ms"] * 1e3, "unit": "µs/step", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
-        **({"o_proj": {"us": r["op_ms"] * 1e3, "weight_bytes": w.d * HD_of(w) * 2,
-                       "gbs": w.d * HD_of(w) * 2 / (r["op_ms"] * 1e-3) / 1e9,
-                       "frac": (w.d * HD_of(w) * 2 / (peaks["hbm_gbs"] * 1e9)) / (r["op_ms"] * 1e-3),
-                       "peak_gbs": peaks["hbm_gbs"]}} if r["op_ms"] is not None else {}),
+        **({"o_proj": o_proj_line(w, r["op_ms"], peaks, args.o_proj_absorbed)} if r["op_ms"] is not None else {}),
         "tensor_core_decode": r["tc"],
         "clocks": r["clocks"],
     }

@@ -183,13 +183,67 @@ mla_status mla_out_proj(const mla_dims *dims, const void *o_lat, const void *W_U
 mla_status mla_o_proj(const mla_dims *dims, const void *o, const void *W_O, int32_t T, void *y, void *ws,
                       size_t ws_bytes, void *stream);
 
+/* W_UV absorbed into the output projection (DeepSeek-V2 explainer, section 3:
+ * the remark that W_UV can be folded into W_O; MLA walk-through, section 1
+ * step 5 and section 3 order B): since o_h = W_UV_h o_lat,h,
+ *   W_OV[r][h*d_c + j] = sum_i W_O[r][h*d_h + i] W_UV[h*d_h + i][j],
+ * a d x n_h*d_c matrix, rounded once to the storage dtype. An offline step:
+ * W_O [d][n_h*d_h], W_UV [n_h*d_h][d_c], W_OV (output) [d][n_h*d_c]. No
+ * workspace. */
+mla_status mla_absorb_wo(const mla_dims *dims, const void *W_O, const void *W_UV, void *W_OV, void *stream);
+
+/* Output projection straight from the latent readout, with W_OV from
+ * mla_absorb_wo: y[t][r] = sum_k W_OV[r][k] o_lat[t][k], k < n_h*d_c (the same
+ * y as mla_out_proj followed by mla_o_proj, up to rounding).
+ *   o_lat [T][n_h][d_c]   W_OV [d][n_h*d_c]   y (output) [T][d]. */
+mla_status mla_o_proj_latent(const mla_dims *dims, const void *o_lat, const void *W_OV, int32_t T, void *y,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* Merged absorption matrix (MLA walk-through, section 3 order B: the merged
+ * matrix can be computed offline): W_UQK_h = W_UK_h^T W_UQ_h, so that
+ * q_lat,h = W_UQK_h c_Q in one product.
+ *   W_UQK[h*d_c + j][c] = sum_i W_UK[h*d_h + i][j] W_UQ[h*d_h + i][c],
+ * n_h*d_c x d_cq, rounded once. W_UQ [n_h*d_h][d_cq], W_UK [n_h*d_h][d_c].
+ * No workspace. */
+mla_status mla_absorb_merge(const mla_dims *dims, const void *W_UQ, const void *W_UK, void *W_UQK, void *stream);
+
+/* mla_absorb_q with the merged matrix: c_Q = W_DQ h_t, q_lat,h = W_UQK_h c_Q,
+ * q_R,h = RoPE(W_QR_h c_Q, positions[t]); same q layout and rounding points
+ * as mla_absorb_q (c_Q rounded once to the storage dtype). */
+mla_status mla_absorb_q_merged(const mla_dims *dims, const void *h, const void *W_DQ, const void *W_UQK,
+                               const void *W_QR, const int32_t *positions, int32_t T, void *q, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* Front end of the step in one call: mla_cache_append and mla_absorb_q over
+ * the same h_t (MLA walk-through, section 1 steps 1 and 3: both paths start
+ * from h_t). On the tensor-core path h is read once, by one weight-streaming
+ * product [W_DKV; W_KR; W_DQ] h whose finalize writes the cache rows and c_Q;
+ * the per-head query chain follows. Results, arguments and error behaviour
+ * are those of the two calls. */
+mla_status mla_front_end(const mla_dims *dims, const void *h, const void *W_DKV, const void *W_KR,
+                         const void *W_DQ, const void *W_UQ, const void *W_QR, const void *W_UK,
+                         const int32_t *seq_idx, const int32_t *positions, int32_t T, const mla_cache *cache,
+                         void *q, void *ws, size_t ws_bytes, void *stream);
+
+/* Self-test of the failure path (no counterpart on the pages). Launches one
+ * small projection kernel whose copy engine is told to issue nothing, so that
+ * its MMA thread's bounded wait runs out after wait_ns nanoseconds; the kernel
+ * then records MLA_ERR_TIMEOUT in the device error word (read it with
+ * mla_get_device_error), frees its tensor memory and returns, with no copy in
+ * flight. The context stays usable. scratch: >= 65536 bytes of device memory,
+ * overwritten. */
+mla_status mla_selftest_timeout(uint64_t wait_ns, void *scratch, size_t scratch_bytes, void *stream);
+
 /* Scratch size in bytes for one call of `op` (MLA_OP_*). `rows` is T for
  * append/absorb/out_proj/o_proj and B for decode; n_q, max_seq_len and
  * num_splits are used by decode only. max_seq_len bounds the tiles of a row
  * for forced splits (0 = unknown: the size then covers num_splits pieces for
  * every row); mla_decode itself requires the size for max_seq_len = the
  * cache's capacity (max_len, or max_blocks_per_seq * block_size). */
-enum { MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3, MLA_OP_O_PROJ = 4 };
+enum {
+  MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3, MLA_OP_O_PROJ = 4,
+  MLA_OP_O_PROJ_LATENT = 5, MLA_OP_ABSORB_MERGED = 6, MLA_OP_FRONT_END = 7, MLA_OP_ABSORB_WO = 8
+};
 size_t mla_workspace_size(const mla_dims *dims, int32_t op, int32_t rows, int32_t n_q,
                           int64_t max_seq_len, int32_t num_splits);
 

@@ -31,15 +31,17 @@ enum Epi : int {
 
 struct Params {
   int m_total;       // rows of D per batch
-  int m_split;       // rows [m_split, m_total) come from the second A map
+  int m_split;       // rows [m_split, m_split2) come from the second A map
+  int m_split2;      // rows [m_split2, m_total) come from the third A map
   int n_total;       // tokens
   int n_tile;        // MMA N (multiple of 16, <= 256)
   int k_total;       // contraction length per batch
   int k_blocks_per_split;
   int splits;
   int a_mn_major;    // A stored with m contiguous (W_UK^T)
+  int b_mn_major;    // B stored with n contiguous (rows are k): n_tile a multiple of 64
   int a_batch_rows;  // A row offset per batch (K-major: m rows; MN-major: k rows)
-  int b_batch_cols;  // B column (k) offset per batch
+  int b_batch_cols;  // B k offset per batch (a column for K-major B, a row for MN-major B)
   int stages;
   float *out;        // EPI_PARTIAL: [batch][split][n_total][m_total]
   int epi;
@@ -51,6 +53,11 @@ struct Params {
   double rope_base;
   const int32_t *positions;
   int prefetch;  // launched with launch overlap: weight boxes of the first stages go out before griddep_wait
+  // failure-path self-test only: every bounded wait gives up after wait_ns
+  // (0: the library's default limit) and, with idle_producer set, the TMA
+  // producer issues nothing, so that the MMA thread's first wait runs out
+  uint64_t wait_ns;
+  int idle_producer;
 };
 
 __host__ __device__ constexpr int b_stage_bytes(int n_tile) { return n_tile * BK * 2; }
@@ -58,7 +65,7 @@ __host__ __device__ constexpr int b_stage_bytes(int n_tile) { return n_tile * BK
 // One CTA: M tile blockIdx.x, N tile blockIdx.y, (batch, split) blockIdx.z.
 __global__ void __launch_bounds__(NUM_THREADS, 2)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
-           const __grid_constant__ CUtensorMap tm_b, const Params p) {
+           const __grid_constant__ CUtensorMap tm_a3, const __grid_constant__ CUtensorMap tm_b, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -71,6 +78,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   const uint32_t done = bars + 8u * (2 * p.stages);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.stages * stage_bytes + 8 * (2 * p.stages + 1));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint64_t wait_ns = p.wait_ns != 0 ? p.wait_ns : MLA_WAIT_NS;
 
   const int m_tile = blockIdx.x, n_tile = blockIdx.y;
   const int batch = blockIdx.z / p.splits, split = blockIdx.z % p.splits;
@@ -97,9 +105,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   if (threadIdx.x == 0) griddep_launch_dependents();
 
   const int m0 = m_tile * BM;
-  const bool second = m0 >= p.m_split;
-  const CUtensorMap *am = second ? &tm_a2 : &tm_a;
-  const int am0 = second ? m0 - p.m_split : m0;
+  const bool third = m0 >= p.m_split2, second = !third && m0 >= p.m_split;
+  const CUtensorMap *am = third ? &tm_a3 : (second ? &tm_a2 : &tm_a);
+  const int am0 = third ? m0 - p.m_split2 : (second ? m0 - p.m_split : m0);
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -121,9 +129,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     };
     auto issue_b = [&](int i) {
       const uint32_t a_dst = stage0 + (i % p.stages) * stage_bytes;
-      tma_load_2d(a_dst + A_STAGE, &tm_b, (kb0 + i) * BK + batch * p.b_batch_cols, n_tile * p.n_tile, full(i % p.stages));
+      if (!p.b_mn_major) {
+        tma_load_2d(a_dst + A_STAGE, &tm_b, (kb0 + i) * BK + batch * p.b_batch_cols, n_tile * p.n_tile, full(i % p.stages));
+      } else {  // B(n, k) at X[k][n]: n_tile / 64 boxes of 64 n x 64 k rows
+        for (int j = 0; j < p.n_tile / 64; ++j)
+          tma_load_2d(a_dst + A_STAGE + j * (64 * BK * 2), &tm_b, n_tile * p.n_tile + 64 * j,
+                      (kb0 + i) * BK + batch * p.b_batch_cols, full(i % p.stages));
+      }
     };
-    const int pre = p.prefetch ? min(nkb, p.stages) : 0;  // stages <= 12: lanes l and 16 + l serve stage l
+    const int nkp = p.idle_producer ? 0 : nkb;  // self-test: nothing is issued, no copy is in flight
+    const int pre = p.prefetch ? min(nkp, p.stages) : 0;  // stages <= 12: lanes l and 16 + l serve stage l
     if (lane == 0)
       for (int i = 0; i < pre; ++i) mbar_arrive_expect_tx(full(i), stage_bytes);
     __syncwarp();
@@ -132,11 +147,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     griddep_wait();
     if (lane < pre) issue_b(lane);
     __syncwarp();
-    for (int i = pre; i < nkb; ++i) {
+    for (int i = pre; i < nkp; ++i) {
       const int s = i % p.stages;
       bool good = true;
       if (lane == 0) {
-        if (i >= p.stages) good = mbar_wait(empty(s), ((i / p.stages) - 1) & 1, abort_flag);
+        if (i >= p.stages) good = mbar_wait(empty(s), ((i / p.stages) - 1) & 1, abort_flag, wait_ns);
         if (good) mbar_arrive_expect_tx(full(s), stage_bytes);
       }
       if (!__shfl_sync(0xffffffffu, good, 0)) break;
@@ -147,10 +162,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = idesc_bf16(BM, p.n_tile, p.a_mn_major != 0, false);
+    const uint32_t idesc = idesc_bf16(BM, p.n_tile, p.a_mn_major != 0, p.b_mn_major != 0);
     for (int i = 0; i < nkb; ++i) {
       const int s = i % p.stages;
-      if (!mbar_wait(full(s), (i / p.stages) & 1, abort_flag)) break;
+      if (!mbar_wait(full(s), (i / p.stages) & 1, abort_flag, wait_ns)) break;
       tc_fence_after();
       const uint32_t a_src = sbase + s * stage_bytes;
       const uint32_t b_src = a_src + A_STAGE;
@@ -158,7 +173,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       for (int kk = 0; kk < BK / 16; ++kk) {
         const uint64_t ad = p.a_mn_major ? sdesc_sw128(a_src + kk * 2048, A_STAGE / 2, 1024)
                                          : sdesc_sw128(a_src + kk * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(b_src + kk * 32, 16, 1024);
+        const uint64_t bd = p.b_mn_major ? sdesc_sw128(b_src + kk * 2048, 64 * BK * 2, 1024)
+                                         : sdesc_sw128(b_src + kk * 32, 16, 1024);
         tc_mma<1>(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
       tc_commit(empty(s));
@@ -169,7 +185,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     const int sp = warp & 3;
     const int row = 32 * sp + lane;  // m within tile
     griddep_wait();  // outputs are written only once the previous kernel has finished
-    mbar_wait_warp(done, 0, abort_flag);
+    mbar_wait_warp(done, 0, abort_flag, wait_ns);
     tc_fence_after();
     const int m = m0 + row;
     const int n_base = n_tile * p.n_tile;
@@ -503,6 +519,40 @@ __global__ void k_fin_append(const float *part, int splits, int T, int d_c, int 
   }
   __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(cache.data) + row * D;
   const float2 x = sum_splits2(part, splits, stride, static_cast<int64_t>(t) * D + e);
+  float x0 = x.x, x1 = x.y;
+  if (e >= d_c) rope_pair(x0, x1, (e - d_c) / 2, d_r, pos, rope_base);
+  *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(x0, x1);
+}
+
+// Finalize of the fused front end: the split sums of the stacked product
+// [W_DKV; W_KR; W_DQ] h (partials [split][T][m_total]). Rows [0, d_c + d_r)
+// are the append (RoPE on [d_c, d_c + d_r), bf16, stored at the cache row of
+// (seq_idx[t], positions[t])); rows [cq_row, cq_row + d_cq) are c_Q (bf16 into
+// cq[t][.]). grid (ceil((d_c + d_r + d_cq) / 256), T), one thread per pair.
+__global__ void k_fin_front(const float *part, int splits, int T, int m_total, int d_c, int d_r, int cq_row,
+                            int d_cq, double rope_base, const int32_t *seq_idx, const int32_t *positions,
+                            CacheView cache, __nv_bfloat16 *cq) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  griddep_wait();
+  const int t = blockIdx.y;
+  const int D = d_c + d_r;
+  const int e = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (e >= D + d_cq) return;
+  const int64_t stride = static_cast<int64_t>(T) * m_total;
+  if (e >= D) {
+    const int c = e - D;
+    const float2 x = sum_splits2(part, splits, stride, static_cast<int64_t>(t) * m_total + cq_row + c);
+    *reinterpret_cast<uint32_t *>(cq + static_cast<int64_t>(t) * d_cq + c) = pack_bf16x2(x.x, x.y);
+    return;
+  }
+  const int pos = positions[t];
+  const int64_t row = cache_row(cache, seq_idx[t], pos);
+  if (row < 0) {
+    if (e == 0) dev_error(MLA_DEVERR_DATA);
+    return;
+  }
+  __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(cache.data) + row * D;
+  const float2 x = sum_splits2(part, splits, stride, static_cast<int64_t>(t) * m_total + e);
   float x0 = x.x, x1 = x.y;
   if (e >= d_c) rope_pair(x0, x1, (e - d_c) / 2, d_r, pos, rope_base);
   *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(x0, x1);

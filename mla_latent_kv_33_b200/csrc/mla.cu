@@ -274,6 +274,74 @@ size_t simt_out_proj_ws(const mla_dims *d, int Tn) {
   return sizeof(float) * static_cast<size_t>(Tn) * d->n_h * d->d_h;
 }
 
+// out(h, a, b) = sum_i L(h, i, a) R(h, i, b), i < d_h, rounded once to T.
+template <typename T>
+void launch_head_product(const void *L, int64_t l_h, int64_t l_i, int64_t l_a, const void *R, int64_t r_h,
+                         int64_t r_i, int64_t r_b, void *out, int64_t o_h, int64_t o_a, int64_t o_b, int A, int Bn,
+                         int I, int H, cudaStream_t st) {
+  dim3 grid((Bn + 255) / 256, A, H);
+  MLA_LAUNCH(mla::k_simt_head_product<T><<<grid, 256, 0, st>>>(static_cast<const T *>(L), l_h, l_i, l_a,
+                                                                static_cast<const T *>(R), r_h, r_i, r_b,
+                                                                static_cast<T *>(out), o_h, o_a, o_b, A, Bn, I));
+}
+
+template <typename T>
+mla_status simt_absorb_wo(const mla_dims *d, const void *W_O, const void *W_UV, void *W_OV, cudaStream_t st) {
+  // W_OV[r][h d_c + j] = sum_i W_O[r][h d_h + i] W_UV[h d_h + i][j]
+  const int64_t HD = static_cast<int64_t>(d->n_h) * d->d_h, HC = static_cast<int64_t>(d->n_h) * d->d_c;
+  launch_head_product<T>(W_O, d->d_h, 1, HD, W_UV, static_cast<int64_t>(d->d_h) * d->d_c, d->d_c, 1, W_OV, d->d_c,
+                         HC, 1, d->d, d->d_c, d->d_h, d->n_h, st);
+  return cuda_check("absorb W_UV into W_O (CUDA cores)");
+}
+
+template <typename T>
+mla_status simt_absorb_merge(const mla_dims *d, const void *W_UQ, const void *W_UK, void *W_UQK, cudaStream_t st) {
+  // W_UQK[h d_c + j][c] = sum_i W_UK[h d_h + i][j] W_UQ[h d_h + i][c]
+  launch_head_product<T>(W_UK, static_cast<int64_t>(d->d_h) * d->d_c, d->d_c, 1, W_UQ,
+                         static_cast<int64_t>(d->d_h) * d->d_cq, d->d_cq, 1, W_UQK,
+                         static_cast<int64_t>(d->d_c) * d->d_cq, d->d_cq, 1, d->d_c, d->d_cq, d->d_h, d->n_h, st);
+  return cuda_check("merged absorption matrix (CUDA cores)");
+}
+
+template <typename T>
+mla_status simt_absorb_q_merged(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQK,
+                                const void *W_QR, const int32_t *positions, int Tn, void *q, void *ws,
+                                cudaStream_t st) {
+  const int64_t HR = static_cast<int64_t>(d->n_h) * d->d_r;
+  const int64_t HC = static_cast<int64_t>(d->n_h) * d->d_c;
+  float *cq = static_cast<float *>(ws);             // [T][d_cq]
+  float *qr = cq + static_cast<int64_t>(Tn) * d->d_cq;  // [T][n_h*d_r]
+  float *ql = qr + Tn * HR;                         // [T][n_h][d_c]
+  launch_linear<T>(static_cast<const T *>(W_DQ), 0, d->d, 1, h, false, 0, d->d, cq, 0, d->d_cq, d->d_cq, d->d, Tn, 1,
+                   st);
+  launch_linear<T>(static_cast<const T *>(W_QR), 0, d->d_cq, 1, cq, true, 0, d->d_cq, qr, 0, HR, static_cast<int>(HR),
+                   d->d_cq, Tn, 1, st);
+  // q_lat,h[j] = sum_c W_UQK[h d_c + j][c] c_Q[c]: batch = head
+  launch_linear<T>(static_cast<const T *>(W_UQK), static_cast<int64_t>(d->d_c) * d->d_cq, d->d_cq, 1, cq, true, 0,
+                   d->d_cq, ql, d->d_c, HC, d->d_c, d->d_cq, Tn, d->n_h, st);
+  MLA_LAUNCH(mla::k_simt_q_store<T><<<Tn * d->n_h, 128, 0, st>>>(ql, qr, d->n_h, d->d_c, d->d_r, d->rope_base,
+                                                                    positions, static_cast<T *>(q)));
+  return cuda_check("merged absorb (CUDA cores)");
+}
+
+size_t simt_absorb_merged_ws(const mla_dims *d, int Tn) {
+  return sizeof(float) * static_cast<size_t>(Tn) * (d->d_cq + static_cast<size_t>(d->n_h) * (d->d_r + d->d_c));
+}
+
+template <typename T>
+mla_status simt_o_proj_latent(const mla_dims *d, const void *o_lat, const void *W_OV, int Tn, void *y, void *ws,
+                              cudaStream_t st) {
+  // y[t][r] = sum_k W_OV[r][k] o_lat[t][k], k < n_h d_c
+  const int64_t HC = static_cast<int64_t>(d->n_h) * d->d_c;
+  float *acc = static_cast<float *>(ws);  // [T][d]
+  launch_linear<T>(static_cast<const T *>(W_OV), 0, HC, 1, o_lat, false, 0, HC, acc, 0, d->d, d->d,
+                   static_cast<int>(HC), Tn, 1, st);
+  const int64_t n = static_cast<int64_t>(Tn) * d->d;
+  const int64_t blocks = (n + 255) / 256;
+  MLA_LAUNCH(mla::k_simt_store<T><<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(acc, static_cast<T *>(y), n));
+  return cuda_check("o_proj (absorbed, CUDA cores)");
+}
+
 
 // ------------------------------------------------------------- TMA maps --
 
@@ -379,11 +447,28 @@ size_t gemm_part_bytes(const GemmShape &g, int T) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const GemmShape &g,
-                       int T, int m_split, bool a_mn_major, int a_batch_rows, int b_batch_cols, G::Params p,
-                       cudaStream_t st) {
+// Operands of one GEMM launch: up to three A maps stacked along m (rows
+// [0, m_split) from a, [m_split, m_split2) from a2, the rest from a3), the B
+// map, their majors and per-batch offsets.
+struct GemmOperands {
+  const CUtensorMap *a, *a2, *a3, *b;
+  int m_split, m_split2;
+  bool a_mn_major, b_mn_major;
+  int a_batch_rows, b_batch_cols;
+};
+
+GemmOperands operands(const CUtensorMap &a, const CUtensorMap &b) {
+  return GemmOperands{&a, &a, &a, &b, 1 << 30, 1 << 30, false, false, 0, 0};
+}
+
+mla_status launch_gemm(const GemmOperands &o, const GemmShape &g, int T, G::Params p, cudaStream_t st) {
+  const int m_split = o.m_split;
+  const bool a_mn_major = o.a_mn_major;
+  const int a_batch_rows = o.a_batch_rows, b_batch_cols = o.b_batch_cols;
   p.m_total = g.m_total;
   p.m_split = m_split;
+  p.m_split2 = o.m_split2;
+  p.b_mn_major = o.b_mn_major ? 1 : 0;
   p.n_total = T;
   p.n_tile = g.n_tile;
   p.k_total = g.k_blocks * G::BK;
@@ -399,7 +484,7 @@ mla_status launch_gemm(const CUtensorMap &ta, const CUtensorMap &ta2, const CUte
                                   "gemm: set shared memory size");
   if (s != MLA_OK) return s;
   dim3 grid(g.m_tiles, g.n_tiles, g.batches * g.splits);
-  return launched(launch_tc(G::k_gemm, grid, dim3(G::NUM_THREADS), smem, st, ta, ta2, tb, p),
+  return launched(launch_tc(G::k_gemm, grid, dim3(G::NUM_THREADS), smem, st, *o.a, *o.a2, *o.a3, *o.b, p),
                   "projection GEMM (tensor cores)");
 }
 
@@ -419,7 +504,10 @@ mla_status tc_append(const mla_dims *d, const void *h, const void *W_DKV, const 
   G::Params p{};
   p.epi = G::EPI_PARTIAL;
   p.out = part;
-  if ((s = launch_gemm(ta, ta2, tb, g, T, d->d_c, false, 0, 0, p, st)) != MLA_OK) return s;
+  GemmOperands op = operands(ta, tb);
+  op.a2 = &ta2;
+  op.m_split = d->d_c;
+  if ((s = launch_gemm(op, g, T, p, st)) != MLA_OK) return s;
   const int D = d->d_c + d->d_r;
   return launched(launch_tc(G::k_fin_append, dim3((D / 2 + 127) / 128, T), dim3(128), 0, st, part, g.splits, T,
                             d->d_c, d->d_r, d->rope_base, seq_idx, positions, view_of(c)),
@@ -444,28 +532,17 @@ AbsorbPlan absorb_plan(const mla_dims *d, int T) {
 
 size_t tc_absorb_ws(const mla_dims *d, int T) { return absorb_plan(d, T).total; }
 
-mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
-                     const void *W_UK, const int32_t *positions, int T, void *q, void *ws, cudaStream_t st) {
+// q = [W_UK_h^T W_UQ_h c_Q | RoPE(W_QR_h c_Q)] from a c_Q already stored (bf16
+// [T][d_cq]): one CTA per head with q_C in shared memory (T <= 128), or
+// [W_UQ; W_QR] then W_UK^T with q_C in the workspace (qc, T * n_h * d_h bf16).
+mla_status tc_absorb_from_cq(const mla_dims *d, const __nv_bfloat16 *cq, const void *W_UQ, const void *W_QR,
+                             const void *W_UK, const int32_t *positions, int T, void *q, __nv_bfloat16 *qc,
+                             cudaStream_t st) {
   const AbsorbPlan a = absorb_plan(d, T);
-  float *part = static_cast<float *>(ws);
-  __nv_bfloat16 *cq = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.cq_off);
-  __nv_bfloat16 *qc = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + a.qc_off);
   const int HD = d->n_h * d->d_h;
   const int64_t Dq = d->d_c + d->d_r;
   CUtensorMap ta, ta2, tb;
   mla_status s;
-  // c_Q = W_DQ h (split K, fp32 partials, then rounded to bf16 for the next product)
-  if ((s = make_tmap_bf16(&ta, W_DQ, d->d, d->d_cq, d->d * 2ull, 64, 128, "W_DQ")) != MLA_OK) return s;
-  if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, a.cq.n_tile, "h")) != MLA_OK) return s;
-  G::Params p{};
-  p.epi = G::EPI_PARTIAL;
-  p.out = part;
-  if ((s = launch_gemm(ta, ta, tb, a.cq, T, d->d_cq, false, 0, 0, p, st)) != MLA_OK) return s;
-  const int64_t pairs = static_cast<int64_t>(T) * d->d_cq / 2;
-  if ((s = launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
-                              dim3(256), 0, st, part, a.cq.splits, T, d->d_cq, cq, static_cast<int64_t>(d->d_cq)),
-                    "c_Q finalize")) != MLA_OK)
-    return s;
   if (a.uq.n_tile <= 128) {
     // one CTA per head: q_C,h = W_UQ_h c_Q, q_R,h = RoPE(W_QR_h c_Q), q_lat,h = W_UK_h^T q_C,h
     CUtensorMap tq, tr, tc, tk;
@@ -499,7 +576,7 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   if ((s = make_tmap_bf16(&ta2, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK)
     return s;
   if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, a.uq.n_tile, "c_Q")) != MLA_OK) return s;
-  p = G::Params{};
+  G::Params p{};
   p.epi = G::EPI_UQ;
   p.dst = qc;
   p.e_split = HD;
@@ -509,7 +586,10 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   p.d_r = d->d_r;
   p.rope_base = d->rope_base;
   p.positions = positions;
-  if ((s = launch_gemm(ta, ta2, tb, a.uq, T, HD, false, 0, 0, p, st)) != MLA_OK) return s;
+  GemmOperands op = operands(ta, tb);
+  op.a2 = &ta2;
+  op.m_split = HD;
+  if ((s = launch_gemm(op, a.uq, T, p, st)) != MLA_OK) return s;
   // q_lat,h = W_UK_h^T q_C,h: A(m = latent j, k = i) = W_UK[h*d_h + i][j], m contiguous
   if ((s = make_tmap_bf16(&ta, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UK")) != MLA_OK) return s;
   if ((s = make_tmap_bf16(&tb, qc, HD, T, HD * 2ull, 64, a.uk.n_tile, "q_C")) != MLA_OK) return s;
@@ -518,7 +598,226 @@ mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const v
   p.dst = static_cast<__nv_bfloat16 *>(q);
   p.e_bs = Dq;
   p.e_ns = d->n_h * Dq;
-  return launch_gemm(ta, ta, tb, a.uk, T, d->d_c, true, d->d_h, d->d_h, p, st);
+  op = operands(ta, tb);
+  op.a_mn_major = true;
+  op.a_batch_rows = d->d_h;
+  op.b_batch_cols = d->d_h;
+  return launch_gemm(op, a.uk, T, p, st);
+}
+
+// c_Q = W_DQ h (split K, fp32 partials, then rounded to bf16 in the workspace).
+mla_status tc_query_latent(const mla_dims *d, const void *h, const void *W_DQ, int T, void *ws, size_t cq_off,
+                           cudaStream_t st) {
+  const GemmShape g = gemm_shape(d->d_cq, T, d->d, 1, true);
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_DQ, d->d, d->d_cq, d->d * 2ull, 64, 128, "W_DQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, g.n_tile, "h")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = static_cast<float *>(ws);
+  if ((s = launch_gemm(operands(ta, tb), g, T, p, st)) != MLA_OK) return s;
+  __nv_bfloat16 *cq = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(ws) + cq_off);
+  const int64_t pairs = static_cast<int64_t>(T) * d->d_cq / 2;
+  return launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
+                            dim3(256), 0, st, static_cast<float *>(ws), g.splits, T, d->d_cq, cq,
+                            static_cast<int64_t>(d->d_cq)),
+                  "c_Q finalize");
+}
+
+mla_status tc_absorb(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                     const void *W_UK, const int32_t *positions, int T, void *q, void *ws, cudaStream_t st) {
+  const AbsorbPlan a = absorb_plan(d, T);
+  mla_status s = tc_query_latent(d, h, W_DQ, T, ws, a.cq_off, st);
+  if (s != MLA_OK) return s;
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  return tc_absorb_from_cq(d, reinterpret_cast<__nv_bfloat16 *>(w8 + a.cq_off), W_UQ, W_QR, W_UK, positions, T, q,
+                           reinterpret_cast<__nv_bfloat16 *>(w8 + a.qc_off), st);
+}
+
+// ---- fused front end: one weight-streaming GEMM over [W_DKV; W_KR; W_DQ] ----
+// Rows of the stacked product: [0, d_c) W_DKV, [d_c, d_c + kr_tiles * 128)
+// W_KR (d_r valid rows, the rest of its tiles zero-filled), then W_DQ.
+struct FrontPlan {
+  GemmShape g;
+  int kr_rows, cq_row;
+  size_t cq_off, qc_off, total;
+};
+
+FrontPlan front_plan(const mla_dims *d, int T) {
+  FrontPlan f;
+  f.kr_rows = (d->d_r + G::BM - 1) / G::BM * G::BM;
+  f.cq_row = d->d_c + f.kr_rows;
+  f.g = gemm_shape(f.cq_row + d->d_cq, T, d->d, 1, true);
+  f.cq_off = align256(gemm_part_bytes(f.g, T));
+  f.qc_off = f.cq_off + align256(static_cast<size_t>(T) * d->d_cq * 2);
+  f.total = f.qc_off + static_cast<size_t>(T) * d->n_h * d->d_h * 2;
+  return f;
+}
+
+size_t tc_front_ws(const mla_dims *d, int T) { return front_plan(d, T).total; }
+
+mla_status tc_front_end(const mla_dims *d, const void *h, const void *W_DKV, const void *W_KR, const void *W_DQ,
+                        const void *W_UQ, const void *W_QR, const void *W_UK, const int32_t *seq_idx,
+                        const int32_t *positions, int T, const mla_cache *c, void *q, void *ws, cudaStream_t st) {
+  const FrontPlan f = front_plan(d, T);
+  CUtensorMap ta, ta2, ta3, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_DKV, d->d, d->d_c, d->d * 2ull, 64, 128, "W_DKV")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&ta2, W_KR, d->d, d->d_r, d->d * 2ull, 64, 128, "W_KR")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&ta3, W_DQ, d->d, d->d_cq, d->d * 2ull, 64, 128, "W_DQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, h, d->d, T, d->d * 2ull, 64, f.g.n_tile, "h")) != MLA_OK) return s;
+  float *part = static_cast<float *>(ws);
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = part;
+  GemmOperands op = operands(ta, tb);
+  op.a2 = &ta2;
+  op.a3 = &ta3;
+  op.m_split = d->d_c;
+  op.m_split2 = f.cq_row;
+  if ((s = launch_gemm(op, f.g, T, p, st)) != MLA_OK) return s;
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  __nv_bfloat16 *cq = reinterpret_cast<__nv_bfloat16 *>(w8 + f.cq_off);
+  const int pairs = (d->d_c + d->d_r + d->d_cq) / 2;
+  if ((s = launched(launch_tc(G::k_fin_front, dim3((pairs + 127) / 128, T), dim3(128), 0, st, part, f.g.splits, T,
+                              f.g.m_total, d->d_c, d->d_r, f.cq_row, d->d_cq, d->rope_base, seq_idx, positions,
+                              view_of(c), cq),
+                    "front-end finalize")) != MLA_OK)
+    return s;
+  return tc_absorb_from_cq(d, cq, W_UQ, W_QR, W_UK, positions, T, q,
+                           reinterpret_cast<__nv_bfloat16 *>(w8 + f.qc_off), st);
+}
+
+// ---- merged-matrix absorption: W_UQK_h = W_UK_h^T W_UQ_h (d_c x d_cq per head) ----
+mla_status tc_absorb_merge(const mla_dims *d, const void *W_UQ, const void *W_UK, void *W_UQK, cudaStream_t st) {
+  // D(m = c, n = j) = sum_i W_UQ[h d_h + i][c] W_UK[h d_h + i][j]: both operands MN-major
+  const GemmShape g = gemm_shape(d->d_cq, d->d_c, d->d_h, d->n_h, false);
+  const int HD = d->n_h * d->d_h;
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 64, "W_UQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UK")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_BF16;
+  p.dst = static_cast<__nv_bfloat16 *>(W_UQK);
+  p.e_bs = static_cast<int64_t>(d->d_c) * d->d_cq;  // head h: rows h d_c ..
+  p.e_ns = d->d_cq;                                  // row j, column c = m
+  GemmOperands op = operands(ta, tb);
+  op.a_mn_major = true;
+  op.b_mn_major = true;
+  op.a_batch_rows = d->d_h;
+  op.b_batch_cols = d->d_h;
+  return launch_gemm(op, g, d->d_c, p, st);
+}
+
+size_t tc_absorb_merged_ws(const mla_dims *d, int T) {
+  const GemmShape cq = gemm_shape(d->d_cq, T, d->d, 1, true);
+  return align256(gemm_part_bytes(cq, T)) + static_cast<size_t>(T) * d->d_cq * 2;
+}
+
+mla_status tc_absorb_q_merged(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQK, const void *W_QR,
+                              const int32_t *positions, int T, void *q, void *ws, cudaStream_t st) {
+  const size_t cq_off = align256(gemm_part_bytes(gemm_shape(d->d_cq, T, d->d, 1, true), T));
+  mla_status s = tc_query_latent(d, h, W_DQ, T, ws, cq_off, st);
+  if (s != MLA_OK) return s;
+  const __nv_bfloat16 *cq = reinterpret_cast<const __nv_bfloat16 *>(static_cast<uint8_t *>(ws) + cq_off);
+  const int64_t Dq = d->d_c + d->d_r;
+  CUtensorMap ta, tb;
+  // q_lat,h = W_UQK_h c_Q: batch = head, A rows h d_c .., bf16 into q[t][h][0 .. d_c)
+  const GemmShape gl = gemm_shape(d->d_c, T, d->d_cq, d->n_h, false);
+  if ((s = make_tmap_bf16(&ta, W_UQK, d->d_cq, static_cast<uint64_t>(d->n_h) * d->d_c, d->d_cq * 2ull, 64, 128,
+                          "W_UQK")) != MLA_OK)
+    return s;
+  if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, gl.n_tile, "c_Q")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_BF16;
+  p.dst = static_cast<__nv_bfloat16 *>(q);
+  p.e_bs = Dq;
+  p.e_ns = d->n_h * Dq;
+  GemmOperands op = operands(ta, tb);
+  op.a_batch_rows = d->d_c;
+  if ((s = launch_gemm(op, gl, T, p, st)) != MLA_OK) return s;
+  // q_R = RoPE(W_QR c_Q): every row of this product is a q_R row
+  const GemmShape gr = gemm_shape(d->n_h * d->d_r, T, d->d_cq, 1, false);
+  if ((s = make_tmap_bf16(&ta, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, gr.n_tile, "c_Q")) != MLA_OK) return s;
+  p = G::Params{};
+  p.epi = G::EPI_UQ;
+  p.e_split = 0;
+  p.q = static_cast<__nv_bfloat16 *>(q);
+  p.n_h = d->n_h;
+  p.d_c = d->d_c;
+  p.d_r = d->d_r;
+  p.rope_base = d->rope_base;
+  p.positions = positions;
+  return launch_gemm(operands(ta, tb), gr, T, p, st);
+}
+
+// ---- W_UV absorbed into the output projection ----
+mla_status tc_absorb_wo(const mla_dims *d, const void *W_O, const void *W_UV, void *W_OV, cudaStream_t st) {
+  // D(m = j, n = r) = sum_i W_UV[h d_h + i][j] W_O[r][h d_h + i]; W_OV[r][h d_c + j]
+  const GemmShape g = gemm_shape(d->d_c, d->d, d->d_h, d->n_h, false);
+  const int HD = d->n_h * d->d_h;
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_UV, d->d_c, HD, d->d_c * 2ull, 64, 64, "W_UV")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, W_O, HD, d->d, HD * 2ull, 64, g.n_tile, "W_O")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_BF16;
+  p.dst = static_cast<__nv_bfloat16 *>(W_OV);
+  p.e_bs = d->d_c;
+  p.e_ns = static_cast<int64_t>(d->n_h) * d->d_c;
+  GemmOperands op = operands(ta, tb);
+  op.a_mn_major = true;
+  op.a_batch_rows = d->d_h;
+  op.b_batch_cols = d->d_h;
+  return launch_gemm(op, g, d->d, p, st);
+}
+
+GemmShape o_proj_latent_shape(const mla_dims *d, int T) { return gemm_shape(d->d, T, d->n_h * d->d_c, 1, true); }
+
+size_t tc_o_proj_latent_ws(const mla_dims *d, int T) { return gemm_part_bytes(o_proj_latent_shape(d, T), T); }
+
+mla_status tc_o_proj_latent(const mla_dims *d, const void *o_lat, const void *W_OV, int T, void *y, void *ws,
+                            cudaStream_t st) {
+  const GemmShape g = o_proj_latent_shape(d, T);
+  const int HC = d->n_h * d->d_c;
+  float *part = static_cast<float *>(ws);
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, W_OV, HC, d->d, HC * 2ull, 64, 128, "W_OV")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, o_lat, HC, T, HC * 2ull, 64, g.n_tile, "o_lat")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = part;
+  if ((s = launch_gemm(operands(ta, tb), g, T, p, st)) != MLA_OK) return s;
+  const int64_t pairs = static_cast<int64_t>(T) * d->d / 2;
+  return launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
+                            dim3(256), 0, st, part, g.splits, T, d->d, static_cast<__nv_bfloat16 *>(y),
+                            static_cast<int64_t>(d->d)),
+                  "o_proj (absorbed) finalize");
+}
+
+// ---- failure-path self-test: a projection GEMM whose producer issues nothing ----
+// The MMA thread's first wait runs out after wait_ns; the kernel records the
+// timeout in the device error word and unwinds (no copy is in flight; tensor
+// memory is freed). scratch: at least SELFTEST_BYTES of device memory.
+constexpr size_t SELFTEST_BYTES = 64 * 1024;
+
+mla_status tc_selftest_timeout(uint64_t wait_ns, void *scratch, cudaStream_t st) {
+  uint8_t *s8 = static_cast<uint8_t *>(scratch);
+  const GemmShape g = gemm_shape(G::BM, 16, G::BK, 1, false);  // one tile: 128 rows, 16 tokens, one K block
+  CUtensorMap ta, tb;
+  mla_status s;
+  if ((s = make_tmap_bf16(&ta, s8, G::BK, G::BM, G::BK * 2ull, 64, 128, "self-test A")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, s8 + 16384, G::BK, 16, G::BK * 2ull, 64, g.n_tile, "self-test B")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_PARTIAL;
+  p.out = reinterpret_cast<float *>(s8 + 32768);
+  p.wait_ns = wait_ns;
+  p.idle_producer = 1;
+  return launch_gemm(operands(ta, tb), g, 16, p, st);
 }
 
 GemmShape out_proj_shape(const mla_dims *d, int T) { return gemm_shape(d->d_h, T, d->d_c, d->n_h, false); }
@@ -538,7 +837,10 @@ mla_status tc_out_proj(const mla_dims *d, const void *o_lat, const void *W_UV, i
   p.dst = static_cast<__nv_bfloat16 *>(o);
   p.e_bs = d->d_h;
   p.e_ns = HD;
-  return launch_gemm(ta, ta, tb, g, T, d->d_h, false, d->d_h, d->d_c, p, st);
+  GemmOperands op = operands(ta, tb);
+  op.a_batch_rows = d->d_h;
+  op.b_batch_cols = d->d_c;
+  return launch_gemm(op, g, T, p, st);
 }
 
 // y = W_O o: split-K over the n_h*d_h columns, fp32 partials, then summed to
@@ -558,7 +860,7 @@ mla_status tc_o_proj(const mla_dims *d, const void *o, const void *W_O, int T, v
   G::Params p{};
   p.epi = G::EPI_PARTIAL;
   p.out = part;
-  if ((s = launch_gemm(ta, ta, tb, g, T, d->d, false, 0, 0, p, st)) != MLA_OK) return s;
+  if ((s = launch_gemm(operands(ta, tb), g, T, p, st)) != MLA_OK) return s;
   const int64_t pairs = static_cast<int64_t>(T) * d->d / 2;
   return launched(launch_tc(G::k_fin_store, dim3(static_cast<int>(std::min<int64_t>(1024, (pairs + 255) / 256))),
                             dim3(256), 0, st, part, g.splits, T, d->d, static_cast<__nv_bfloat16 *>(y),
@@ -785,7 +1087,7 @@ int32_t mla_get_launch_overlap(void) { return g_overlap.load(std::memory_order_r
 
 int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   if (d == nullptr || !tc_geometry(d)) return 0;
-  return (op >= MLA_OP_APPEND && op <= MLA_OP_O_PROJ) ? 1 : 0;
+  return (op >= MLA_OP_APPEND && op <= MLA_OP_ABSORB_WO) ? 1 : 0;
 }
 
 size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len,
@@ -799,6 +1101,10 @@ size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n
       return tc ? mla::decode_tc_ws(rows, n_q < 1 ? 1 : n_q, sm_count(), num_splits, max_seq_len) : 0;
     case MLA_OP_OUT_PROJ: return tc ? tc_out_proj_ws(d, rows) : simt_out_proj_ws(d, rows);
     case MLA_OP_O_PROJ: return tc ? tc_o_proj_ws(d, rows) : simt_o_proj_ws(d, rows);
+    case MLA_OP_O_PROJ_LATENT: return tc ? tc_o_proj_latent_ws(d, rows) : simt_o_proj_ws(d, rows);
+    case MLA_OP_ABSORB_MERGED: return tc ? tc_absorb_merged_ws(d, rows) : simt_absorb_merged_ws(d, rows);
+    case MLA_OP_FRONT_END:
+      return tc ? tc_front_ws(d, rows) : std::max(simt_append_ws(d, rows), simt_absorb_ws(d, rows));
   }
   return 0;
 }
@@ -923,6 +1229,99 @@ mla_status mla_o_proj(const mla_dims *d, const void *o, const void *W_O, int32_t
   if (tc_geometry(d)) return tc_o_proj(d, o, W_O, T, y, ws, st);
   if (d->dtype == MLA_BF16) return simt_o_proj<__nv_bfloat16>(d, o, W_O, T, y, ws, st);
   return simt_o_proj<float>(d, o, W_O, T, y, ws, st);
+}
+
+mla_status mla_absorb_wo(const mla_dims *d, const void *W_O, const void *W_UV, void *W_OV, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (!W_O || !W_UV || !W_OV) return fail(MLA_ERR_INVALID_ARG, "absorb_wo: NULL tensor argument");
+  if (!aligned16(W_O) || !aligned16(W_UV) || !aligned16(W_OV))
+    return fail(MLA_ERR_INVALID_ARG, "absorb_wo: tensors must be 16-byte aligned");
+  if (d->d > 65535) return fail(MLA_ERR_UNSUPPORTED, "absorb_wo: d > 65535");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_absorb_wo(d, W_O, W_UV, W_OV, st);
+  if (d->dtype == MLA_BF16) return simt_absorb_wo<__nv_bfloat16>(d, W_O, W_UV, W_OV, st);
+  return simt_absorb_wo<float>(d, W_O, W_UV, W_OV, st);
+}
+
+mla_status mla_o_proj_latent(const mla_dims *d, const void *o_lat, const void *W_OV, int32_t T, void *y, void *ws,
+                             size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!o_lat || !W_OV || !y) return fail(MLA_ERR_INVALID_ARG, "o_proj_latent: NULL tensor argument");
+  if (!aligned16(o_lat) || !aligned16(W_OV) || !aligned16(y))
+    return fail(MLA_ERR_INVALID_ARG, "o_proj_latent: tensors must be 16-byte aligned");
+  if (d->d % 2 != 0) return fail(MLA_ERR_UNSUPPORTED, "o_proj_latent: d must be even");
+  const size_t need = mla_workspace_size(d, MLA_OP_O_PROJ_LATENT, T, 1, 0, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "o_proj_latent needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_o_proj_latent(d, o_lat, W_OV, T, y, ws, st);
+  if (d->dtype == MLA_BF16) return simt_o_proj_latent<__nv_bfloat16>(d, o_lat, W_OV, T, y, ws, st);
+  return simt_o_proj_latent<float>(d, o_lat, W_OV, T, y, ws, st);
+}
+
+mla_status mla_absorb_merge(const mla_dims *d, const void *W_UQ, const void *W_UK, void *W_UQK, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (!W_UQ || !W_UK || !W_UQK) return fail(MLA_ERR_INVALID_ARG, "absorb_merge: NULL tensor argument");
+  if (!aligned16(W_UQ) || !aligned16(W_UK) || !aligned16(W_UQK))
+    return fail(MLA_ERR_INVALID_ARG, "absorb_merge: tensors must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_absorb_merge(d, W_UQ, W_UK, W_UQK, st);
+  if (d->dtype == MLA_BF16) return simt_absorb_merge<__nv_bfloat16>(d, W_UQ, W_UK, W_UQK, st);
+  return simt_absorb_merge<float>(d, W_UQ, W_UK, W_UQK, st);
+}
+
+mla_status mla_absorb_q_merged(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQK,
+                               const void *W_QR, const int32_t *positions, int32_t T, void *q, void *ws,
+                               size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!h || !W_DQ || !W_UQK || !W_QR || !positions || !q)
+    return fail(MLA_ERR_INVALID_ARG, "absorb_q_merged: NULL tensor argument");
+  if (!aligned16(h) || !aligned16(W_DQ) || !aligned16(W_UQK) || !aligned16(W_QR) || !aligned16(q))
+    return fail(MLA_ERR_INVALID_ARG, "absorb_q_merged: tensors must be 16-byte aligned");
+  const size_t need = mla_workspace_size(d, MLA_OP_ABSORB_MERGED, T, 1, 0, 0);
+  if (ws_bytes < need || (need && !ws))
+    return fail(MLA_ERR_WORKSPACE, "absorb_q_merged needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_absorb_q_merged(d, h, W_DQ, W_UQK, W_QR, positions, T, q, ws, st);
+  if (d->dtype == MLA_BF16)
+    return simt_absorb_q_merged<__nv_bfloat16>(d, h, W_DQ, W_UQK, W_QR, positions, T, q, ws, st);
+  return simt_absorb_q_merged<float>(d, h, W_DQ, W_UQK, W_QR, positions, T, q, ws, st);
+}
+
+mla_status mla_front_end(const mla_dims *d, const void *h, const void *W_DKV, const void *W_KR, const void *W_DQ,
+                         const void *W_UQ, const void *W_QR, const void *W_UK, const int32_t *seq_idx,
+                         const int32_t *positions, int32_t T, const mla_cache *c, void *q, void *ws, size_t ws_bytes,
+                         void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!h || !W_DKV || !W_KR || !W_DQ || !W_UQ || !W_QR || !W_UK || !seq_idx || !positions || !q)
+    return fail(MLA_ERR_INVALID_ARG, "front_end: NULL tensor argument");
+  if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(W_KR) || !aligned16(W_DQ) || !aligned16(W_UQ) ||
+      !aligned16(W_QR) || !aligned16(W_UK) || !aligned16(q))
+    return fail(MLA_ERR_INVALID_ARG, "front_end: tensors must be 16-byte aligned");
+  if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
+  const size_t need = mla_workspace_size(d, MLA_OP_FRONT_END, T, 1, 0, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "front_end needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d))
+    return tc_front_end(d, h, W_DKV, W_KR, W_DQ, W_UQ, W_QR, W_UK, seq_idx, positions, T, c, q, ws, st);
+  // CUDA-core dims: the two calls one after the other (each reads h)
+  if ((s = mla_cache_append(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, ws_bytes, stream)) != MLA_OK) return s;
+  return mla_absorb_q(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, ws_bytes, stream);
+}
+
+mla_status mla_selftest_timeout(uint64_t wait_ns, void *scratch, size_t scratch_bytes, void *stream) {
+  if (wait_ns == 0) return fail(MLA_ERR_INVALID_ARG, "selftest_timeout: wait_ns must be positive");
+  if (scratch == nullptr || !aligned16(scratch) || scratch_bytes < SELFTEST_BYTES)
+    return fail(MLA_ERR_INVALID_ARG, "selftest_timeout: needs %zu bytes of 16-byte aligned device scratch",
+                SELFTEST_BYTES);
+  return tc_selftest_timeout(wait_ns, scratch, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -100,8 +100,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete. `abort` is a
 // per-CTA shared flag: once any role of this CTA gives up, the others stop
-// waiting too. Returns false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
+// waiting too. Returns false on timeout (limit_ns of %globaltimer) or abort.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = MLA_WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   if (abort != nullptr && *abort) return false;
   const uint64_t t0 = globaltimer_ns();
@@ -109,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > MLA_WAIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         dev_error(MLA_DEVERR_TIMEOUT);
         if (abort != nullptr) *abort = 1;
         return false;
@@ -120,8 +121,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // All 32 lanes wait; the result is made warp-uniform so that the
 // warp-collective tcgen05.ld/st that follow always run converged.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort,
+                                               uint64_t limit_ns = MLA_WAIT_NS) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -31,6 +31,26 @@ __global__ void __launch_bounds__(256) k_simt_linear(const TW *__restrict__ W, i
   if (lane == 0) Y[bt * y_sb + t * y_st + n] = acc;
 }
 
+// Per-head product of two matrices that share their row index i (d_h rows per
+// head): out(h, a, b) = sum_i L(h, i, a) R(h, i, b), rounded once to the
+// storage type. X(h, i, c) = X[h*s_h + i*s_i + c*s_c] for L, R and out (whose
+// i stride is unused). One thread per output element; grid (ceil(B/256), A, H).
+template <typename T>
+__global__ void __launch_bounds__(256) k_simt_head_product(const T *__restrict__ L, int64_t l_h, int64_t l_i,
+                                                           int64_t l_a, const T *__restrict__ R, int64_t r_h,
+                                                           int64_t r_i, int64_t r_b, T *__restrict__ out,
+                                                           int64_t o_h, int64_t o_a, int64_t o_b, int A, int Bn,
+                                                           int I) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  const int a = blockIdx.y, h = blockIdx.z;
+  if (b >= Bn || a >= A) return;
+  const T *l = L + h * l_h + a * l_a;
+  const T *r = R + h * r_h + b * r_b;
+  float acc = 0.f;
+  for (int i = 0; i < I; ++i) acc += ld_f(l + i * l_i) * ld_f(r + i * r_i);
+  out[h * o_h + a * o_a + b * o_b] = from_f<T>(acc);
+}
+
 // Append epilogue: rows [T][D] fp32 -> RoPE on [d_c, D) at positions[t] ->
 // storage dtype -> cache row of (seq_idx[t], positions[t]). One block per t.
 template <typename T>

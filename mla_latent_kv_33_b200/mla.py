@@ -23,7 +23,8 @@ _lib = C.CDLL(LIB_PATH)
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA, MLA_ERR_TIMEOUT, \
     MLA_ERR_DEVICE_DATA = range(7)
 MLA_BF16, MLA_FP32 = 0, 1
-OP_APPEND, OP_ABSORB, OP_DECODE, OP_OUT_PROJ, OP_O_PROJ = range(5)
+OP_APPEND, OP_ABSORB, OP_DECODE, OP_OUT_PROJ, OP_O_PROJ, OP_O_PROJ_LATENT, OP_ABSORB_MERGED, OP_FRONT_END, \
+    OP_ABSORB_WO = range(9)
 
 
 class Dims(C.Structure):
@@ -47,6 +48,13 @@ _lib.mla_decode.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_i
 _lib.mla_out_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
 _lib.mla_o_proj.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
 _lib.mla_decode_noalloc.argtypes = [C.POINTER(Dims), _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P, _P, _P]
+_lib.mla_absorb_wo.argtypes = [C.POINTER(Dims), _P, _P, _P, _P]
+_lib.mla_o_proj_latent.argtypes = [C.POINTER(Dims), _P, _P, C.c_int32, _P, _P, _S, _P]
+_lib.mla_absorb_merge.argtypes = [C.POINTER(Dims), _P, _P, _P, _P]
+_lib.mla_absorb_q_merged.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, C.c_int32, _P, _P, _S, _P]
+_lib.mla_front_end.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_int32,
+                               C.POINTER(CacheDesc), _P, _P, _S, _P]
+_lib.mla_selftest_timeout.argtypes = [C.c_uint64, _P, _S, _P]
 _lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_int32]
 _lib.mla_workspace_size.restype = C.c_size_t
 _lib.mla_get_device_error.argtypes = [_P]
@@ -57,7 +65,8 @@ _lib.mla_uses_tensor_cores.argtypes = [C.POINTER(Dims), C.c_int32]
 _lib.mla_uses_tensor_cores.restype = C.c_int32
 _lib.mla_kernel_launches.restype = C.c_uint64
 for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj", "mla_o_proj",
-           "mla_get_device_error", "mla_set_launch_overlap", "mla_get_launch_overlap"):
+           "mla_get_device_error", "mla_set_launch_overlap", "mla_get_launch_overlap", "mla_absorb_wo",
+           "mla_o_proj_latent", "mla_absorb_merge", "mla_absorb_q_merged", "mla_front_end", "mla_selftest_timeout"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -175,6 +184,46 @@ def mla_o_proj(p: Dims, o, W_O, y, ws=None, stream=None):
     ws, nbytes = _ws(p, OP_O_PROJ, T, 1, ws)
     _check(_lib.mla_o_proj(C.byref(p), _ptr(o), _ptr(W_O), T, _ptr(y), _ptr(ws), nbytes, _stream(stream)),
            "mla_o_proj")
+
+
+def mla_absorb_wo(p: Dims, W_O, W_UV, W_OV, stream=None):
+    """W_OV[r][h d_c + j] = sum_i W_O[r][h d_h + i] W_UV[h d_h + i][j] (offline)."""
+    _check(_lib.mla_absorb_wo(C.byref(p), _ptr(W_O), _ptr(W_UV), _ptr(W_OV), _stream(stream)), "mla_absorb_wo")
+
+
+def mla_o_proj_latent(p: Dims, o_lat, W_OV, y, ws=None, stream=None):
+    T = o_lat.shape[0]
+    ws, nbytes = _ws(p, OP_O_PROJ_LATENT, T, 1, ws)
+    _check(_lib.mla_o_proj_latent(C.byref(p), _ptr(o_lat), _ptr(W_OV), T, _ptr(y), _ptr(ws), nbytes,
+                                  _stream(stream)), "mla_o_proj_latent")
+
+
+def mla_absorb_merge(p: Dims, W_UQ, W_UK, W_UQK, stream=None):
+    """W_UQK[h d_c + j][c] = sum_i W_UK[h d_h + i][j] W_UQ[h d_h + i][c] (offline)."""
+    _check(_lib.mla_absorb_merge(C.byref(p), _ptr(W_UQ), _ptr(W_UK), _ptr(W_UQK), _stream(stream)),
+           "mla_absorb_merge")
+
+
+def mla_absorb_q_merged(p: Dims, h, W_DQ, W_UQK, W_QR, positions, q, ws=None, stream=None):
+    T = h.shape[0]
+    ws, nbytes = _ws(p, OP_ABSORB_MERGED, T, 1, ws)
+    _check(_lib.mla_absorb_q_merged(C.byref(p), _ptr(h), _ptr(W_DQ), _ptr(W_UQK), _ptr(W_QR), _ptr(positions), T,
+                                    _ptr(q), _ptr(ws), nbytes, _stream(stream)), "mla_absorb_q_merged")
+
+
+def mla_front_end(p: Dims, h, W_DKV, W_KR, W_DQ, W_UQ, W_QR, W_UK, seq_idx, positions, cache: Cache, q, ws=None,
+                  stream=None):
+    T = h.shape[0]
+    ws, nbytes = _ws(p, OP_FRONT_END, T, 1, ws)
+    _check(_lib.mla_front_end(C.byref(p), _ptr(h), _ptr(W_DKV), _ptr(W_KR), _ptr(W_DQ), _ptr(W_UQ), _ptr(W_QR),
+                              _ptr(W_UK), _ptr(seq_idx), _ptr(positions), T, C.byref(cache.desc), _ptr(q), _ptr(ws),
+                              nbytes, _stream(stream)), "mla_front_end")
+
+
+def mla_selftest_timeout(wait_ns: int, scratch, stream=None):
+    """Launch the failure-path self-test (a kernel whose bounded wait runs out)."""
+    _check(_lib.mla_selftest_timeout(int(wait_ns), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                     _stream(stream)), "mla_selftest_timeout")
 
 
 def mla_get_device_error(stream=None) -> int:

@@ -160,7 +160,7 @@ def test_workspace_sizes(m):
     assert ws(m.OP_DECODE, 64, 2) > ws(m.OP_DECODE, 64, 1)
     assert ws(m.OP_DECODE, 0) == 0 and ws(m.OP_APPEND, -1) == 0
     assert m._lib.mla_workspace_size(None, m.OP_DECODE, 64, 1, 0, 0) == 0
-    assert ws(7, 64) == 0  # unknown op
+    assert ws(99, 64) == 0  # unknown op
 
 
 def test_tensor_core_geometry_switch(m):
@@ -181,3 +181,38 @@ def test_python_binding_raises_with_status_and_message(m):
         m.mla_absorb_q(d, h, h, h, h, h, torch.zeros(0, dtype=torch.int32), h, ws=None, stream=NoStream())
     assert e.value.status == m.MLA_ERR_INVALID_ARG
     assert "T must be positive" in str(e.value)
+
+
+def test_next_row_entry_points_validate_before_any_launch(m):
+    d = v2(m)
+    c = paged_cache(m)
+    L = m._lib
+    # NULL tensors
+    assert L.mla_absorb_wo(C.byref(d), None, A, A, None) == m.MLA_ERR_INVALID_ARG
+    assert L.mla_absorb_merge(C.byref(d), A, None, A, None) == m.MLA_ERR_INVALID_ARG
+    assert L.mla_o_proj_latent(C.byref(d), A, A, 4, None, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
+    # misaligned, non-positive T, too little workspace
+    assert L.mla_absorb_wo(C.byref(d), MIS, A, A, None) == m.MLA_ERR_INVALID_ARG and "aligned" in last_msg(m)
+    assert L.mla_o_proj_latent(C.byref(d), A, A, 0, A, A, 1 << 30, None) == m.MLA_ERR_INVALID_ARG
+    need = L.mla_workspace_size(C.byref(d), m.OP_O_PROJ_LATENT, 8, 1, 0, 0)
+    assert need > 0 and L.mla_o_proj_latent(C.byref(d), A, A, 8, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
+    need = L.mla_workspace_size(C.byref(d), m.OP_ABSORB_MERGED, 8, 1, 0, 0)
+    assert need > 0
+    assert L.mla_absorb_q_merged(C.byref(d), A, A, A, A, A, 8, A, A, need - 1, None) == m.MLA_ERR_WORKSPACE
+    assert L.mla_absorb_q_merged(C.byref(d), A, A, A, A, None, 8, A, A, need, None) == m.MLA_ERR_INVALID_ARG
+    need = L.mla_workspace_size(C.byref(d), m.OP_FRONT_END, 8, 1, 0, 0)
+    # the fused front end needs at least what the append and the absorb need
+    assert need >= L.mla_workspace_size(C.byref(d), m.OP_ABSORB, 8, 1, 0, 0)
+    assert L.mla_front_end(C.byref(d), A, A, A, A, A, A, A, A, A, 8, C.byref(c), A, A, need - 1,
+                           None) == m.MLA_ERR_WORKSPACE
+    assert L.mla_front_end(C.byref(d), A, A, A, A, A, A, A, A, A, 0, C.byref(c), A, A, need,
+                           None) == m.MLA_ERR_INVALID_ARG
+    bad = paged_cache(m, block_table=None)
+    assert L.mla_front_end(C.byref(d), A, A, A, A, A, A, A, A, A, 8, C.byref(bad), A, A, need,
+                           None) == m.MLA_ERR_INVALID_ARG and "block_table" in last_msg(m)
+    # the self-test needs a positive limit and 64 KiB of aligned scratch
+    assert L.mla_selftest_timeout(0, A, 65536, None) == m.MLA_ERR_INVALID_ARG
+    assert L.mla_selftest_timeout(1000, A, 65535, None) == m.MLA_ERR_INVALID_ARG
+    assert L.mla_selftest_timeout(1000, MIS, 65536, None) == m.MLA_ERR_INVALID_ARG
+    # every new op is served by the tensor cores at DeepSeek dims
+    assert all(L.mla_uses_tensor_cores(C.byref(d), op) == 1 for op in range(9))
