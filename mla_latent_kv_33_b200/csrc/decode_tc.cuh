@@ -550,61 +550,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     }
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    // The tensor pipe retires a pair M128 x N256 x K16 instruction in ~40 ns;
-    // the issuing thread must not take longer than that per instruction. So
-    // every item is issued from fully unrolled code with compile-time slot
-    // indices, K offsets and accumulate flags, and descriptors are formed by
-    // adding constants to per-slot bases built once (the 14-bit start address
-    // field counts 16-byte units; a 32-byte K step adds 2, and no address
-    // here comes near the field's 256 KB limit).
-    // Ring groups always start at big slot 0 (every piece and every tile uses
-    // the big slots in groups of four), so score item q of a tile sits in big
-    // slot q (q < 4) or the small slot (q = 4), and value item (vp, j) in big
-    // slot 2 vp + j; a big slot's fill parity is the group count's parity.
     if (rank == 0 && lane == 0) {
       PieceIter it = it0;
       Piece pc{};
-      int gi = 0, grp = 0, nsmall = 0, gz = 0, npc = 0;
+      int gi = 0, nbig = 0, nsmall = 0, gz = 0, npc = 0, empty_bar = 0;
       bool ok = true;
-      const uint64_t dq = sdesc_sw128(sbase + OFF_Q, 16, 1024);
-      const uint64_t dks = sdesc_sw128(sbase + OFF_SMALL, 16, 1024);
-      uint64_t dk[NBIG], dv[NBIG];
-#pragma unroll
-      for (int sl = 0; sl < NBIG; ++sl) {
-        dk[sl] = sdesc_sw128(sbase + OFF_BIG + sl * BIG, 16, 1024);
-        dv[sl] = sdesc_sw128(sbase + OFF_BIG + sl * BIG, ATOM, HALF);
-      }
+      auto take = [&](bool big) -> uint32_t {  // next ring item in consumption order, once it has landed
+        int slot, use;
+        if (big) {
+          slot = nbig % NBIG;
+          use = nbig / NBIG;
+          ++nbig;
+        } else {
+          slot = 0;
+          use = nsmall++;
+        }
+        empty_bar = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
+        if (!mbar_wait(bar(big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL), use & 1, abort_flag)) return 0;
+        tc_fence_after();
+        return sbase + (big ? OFF_BIG + slot * BIG : OFF_SMALL);
+      };
+      auto release = [&]() { tc_commit_pair(bar(empty_bar), 0x3); };
       // PV of global tile gt (tile ti of the current piece): A = P in tensor
       // memory; K step m of value item (vp, j) takes 8 tokens of block vp and 8
       // of block vp + 2 (one B descriptor over both halves of the item)
       auto issue_pv = [&](int gt, int ti, bool first) -> bool {
         const int zc = partial_chunk(pc.vis, ti);
         const uint32_t p_col = tmem + S_COL + 128 * (gt & 1);
-        const uint32_t par = grp & 1;
+        for (int vp = 0; vp < 2; ++vp)
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t vb = take(true);
+            if (vb == 0) return false;
+            if (vp == 0 && j == 0) {
+              if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
+              if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+              tc_fence_after();
+            }
+            if (zc >= 0 && vp == (zc & 1)) {  // both CTAs zero the rows past the end first
+              mbar_arrive(bar(BAR_V_LANDED));
+              mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
+              if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
+              ++gz;
+              tc_fence_after();
+            }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int vp = g >> 1, j = g & 1;
-          if (!mbar_wait(bar(BAR_BIG_FULL + g), par, abort_flag)) return false;
-          if (g == 0) {
-            if (!mbar_wait(bar(BAR_P_FULL), gt & 1, abort_flag)) return false;
-            if (first && npc > 0 && !mbar_wait(bar(BAR_O_FREE), (npc - 1) & 1, abort_flag)) return false;
+            for (int m = 0; m < 8; ++m)
+              tc_mma_ts<2>(tmem + 128 * j, p_col + 8 * (8 * vp + m), sdesc_sw128(vb + m * 1024, ATOM, HALF), IDESC_PV,
+                           (first && vp == 0 && m == 0) ? 0u : 1u);
+            release();
           }
-          tc_fence_after();
-          if (zc >= 0 && vp == (zc & 1)) {  // both CTAs zero the rows past the end first
-            mbar_arrive(bar(BAR_V_LANDED));
-            mbar_arrive_cluster(mapa_shared(bar(BAR_V_LANDED), 1));
-            if (!mbar_wait(bar(BAR_ZERO_DONE), gz & 1, abort_flag)) return false;
-            ++gz;
-            tc_fence_after();
-          }
-          const uint32_t acc0 = (first && vp == 0) ? 0u : 1u;
-#pragma unroll
-          for (int m = 0; m < 8; ++m)
-            tc_mma_ts<2>(tmem + 128 * j, p_col + 8 * (8 * vp + m), dv[g] + static_cast<uint64_t>(m * (1024 >> 4)),
-                         IDESC_PV, m == 0 ? acc0 : 1u);
-          tc_commit_pair(bar(BAR_BIG_EMPTY + g), 0x3);
-        }
-        ++grp;
         tc_commit_pair(bar(BAR_O_FULL), 0x3);
         return true;
       };
@@ -612,30 +606,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         if (!mbar_wait(bar(BAR_Q_FULL), npc & 1, abort_flag)) break;
         const int n = pc.t_end - pc.t_begin;
         for (int i = 0; i < n && ok; ++i, ++gi) {
-          const uint32_t d = tmem + S_COL + 128 * (gi & 1);  // S(gi) goes over P(gi - 2), read by PV(gi - 2) before it
-          const uint32_t par = grp & 1;
-#pragma unroll
+          const int b = gi & 1;  // S(gi) goes over P(gi - 2), read by PV(gi - 2), issued before it
           for (int q = 0; q < K_ITEMS; ++q) {
             const bool big = q < K_ITEMS - 1;
-            if (!mbar_wait(bar(big ? BAR_BIG_FULL + q : BAR_SMALL_FULL), big ? par : (nsmall & 1), abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t db = big ? dk[q] : dks;
+            const uint32_t kbuf = take(big);
+            if (kbuf == 0) { ok = false; break; }
 #pragma unroll
-            for (int c = 0; c < (big ? 2 : 1); ++c)
+            for (int c = 0; c < 2; ++c) {
+              if (!big && c == 1) break;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                tc_mma<2>(d, dq + static_cast<uint64_t>(((2 * q + c) * CHUNK_Q + kk * 32) >> 4),
-                          db + static_cast<uint64_t>((c * CHUNK_K + kk * 32) >> 4), IDESC_S,
-                          (q > 0 || c > 0 || kk > 0) ? 1u : 0u);
-            tc_commit_pair(bar(big ? BAR_BIG_EMPTY + q : BAR_SMALL_EMPTY), 0x3);
+                tc_mma<2>(tmem + S_COL + 128 * b, sdesc_sw128(sbase + OFF_Q + (2 * q + c) * CHUNK_Q + kk * 32, 16, 1024),
+                          sdesc_sw128(kbuf + c * CHUNK_K + kk * 32, 16, 1024), IDESC_S, (q > 0 || c > 0 || kk > 0) ? 1u : 0u);
+            }
+            release();
           }
           if (!ok) break;
-          ++grp;
-          ++nsmall;
-          tc_commit_pair(bar(BAR_S_FULL + (gi & 1)), 0x3);
+          tc_commit_pair(bar(BAR_S_FULL + b), 0x3);
           if (i == n - 1) tc_commit_pair(bar(BAR_Q_EMPTY), 0x3);
           if (i > 0 && !issue_pv(gi - 1, pc.t_begin + i - 1, i == 1)) { ok = false; break; }
         }
@@ -667,31 +654,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         mbar_wait_warp(bar(BAR_S_FULL + b), (gi >> 1) & 1, abort_flag);
         tc_fence_after();
         const uint32_t s_addr = lane_addr + S_COL + 128 * b;
-        // the thread's 128 scores, loaded at once and kept in registers for
-        // both passes; scores of tokens past the visible end become -inf
-        uint32_t sr[128];
-        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        tmem_wait_ld();
-        if (vis_t - tok0 < OWN) {
+        // pass 1: row max over this thread's 128 tokens, then with the partner lane
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t sr[32];
+          tmem_ld32(s_addr + 32 * q4, sr);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < OWN; ++c)
-            if (tok0 + c >= vis_t) sr[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 32; ++c)
+            if (tok0 + 32 * q4 + c < vis_t) mx = fmaxf(mx, __uint_as_float(sr[c]));
         }
-        // pass 1: row max over this thread's 128 tokens, then with the partner
-        // lane (L ^ 64, in warp sp ^ 2): only the two partner warps synchronise
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < OWN; c += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        }
-        float mx = fmaxf(mx0, mx1);
-        const uint32_t pair_bar = 2 + (sp & 1);
         red[(gi & 1) * 128 + L] = mx;
-        named_bar_sync(pair_bar, 64);
+        named_bar_sync(1, 128);
         mx = fmaxf(mx, red[(gi & 1) * 128 + (L ^ 64)]);
         bool rescale = false;
         float alpha = 1.f;
@@ -709,26 +684,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         // K groups 4 q4 .. 4 q4 + 3; a group is 8 tokens of each half of the tile,
         // the first half in columns 8 g + 0..3 and the second in 8 g + 4..7, in
         // both lanes of the row. The partner lane (L ^ 64) holds the other half.
-        // The exchange buffer holds 16 words per thread: one chunk per round,
-        // a partner-pair barrier after the writes and one before the reuse.
         const float mo = m_ref * c2;
-        float ps0 = 0.f, ps1 = 0.f;
+        float ps = 0.f;
         uint4 *xb = reinterpret_cast<uint4 *>(smem + OFF_XBUF);
-#pragma unroll
+#pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t sr[32];
+          tmem_ld32(s_addr + 32 * q4, sr);
+          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[32 * q4 + 2 * c]), c2, -mo));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[32 * q4 + 2 * c + 1]), c2, -mo));
-            ps0 += p0;
-            ps1 += p1;
+            const int t = tok0 + 32 * q4 + 2 * c;
+            const float p0 = t < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c]), c2, -mo)) : 0.f;
+            const float p1 = t + 1 < vis_t ? ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), c2, -mo)) : 0.f;
+            ps += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }
-          if (q4 > 0) named_bar_sync(pair_bar, 64);  // the partner has read the previous chunk
 #pragma unroll
           for (int u = 0; u < 4; ++u) xb[L * 4 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          named_bar_sync(pair_bar, 64);
+          named_bar_sync(1, 128);
           uint32_t pw[32];
 #pragma unroll
           for (int gg = 0; gg < 4; ++gg) {
@@ -742,14 +717,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
             }
           }
           tmem_st32(s_addr + 32 * q4, pw);
+          named_bar_sync(1, 128);  // the exchange buffer is reused by the next chunk
         }
-        named_bar_sync(pair_bar, 64);  // the exchange buffer is free for the next tile
-        const float ps = ps0 + ps1;
         tmem_wait_st();
-        // P is released only after the previous tile's PV has finished: O may
-        // be rescaled, and the MMA thread has then consumed the previous P_FULL
-        // phase, so that this arrival can never run two phases ahead of its
-        // parity wait.
+        // O is rescaled only after the previous tile's PV has finished with it
         if (gi > 0) mbar_wait_warp(bar(BAR_O_FULL), (gi - 1) & 1, abort_flag);
         tc_fence_after();
         if (rescale) {
