@@ -81,7 +81,14 @@ def parse():
                     help="append and absorb in one call (mla_front_end: h read once) instead of two calls on two streams")
     ap.add_argument("--merged-absorb", action="store_true",
                     help="absorb with the merged matrix W_UK_h^T W_UQ_h (mla_absorb_q_merged)")
+    ap.add_argument("--order-a", action="store_true",
+                    help="attention in order A (mla_query_heads + mla_attend_order_a: decompress K/V per head, then "
+                         "192-d attention) in place of absorb + decode + W_UV readout; default workload v2_prefill_c512")
     a = ap.parse_args()
+    if a.order_a and (a.fused_front_end or a.merged_absorb or a.with_o_proj or a.num_splits):
+        ap.error("--order-a replaces the absorb, the decode and the readout: no other path option applies")
+    if a.order_a and "--workload" not in sys.argv:
+        a.workload = "v2_prefill_c512"
     if a.o_proj_absorbed and not a.with_o_proj:
         ap.error("--o-proj-absorbed needs --with-o-proj")
     if a.merged_absorb and a.fused_front_end:
@@ -251,12 +258,19 @@ def run_ours(args, rank, world, local_rank):
     out_key = "y" if args.with_o_proj else "o"  # what a step hands back to the host
     o = bufs[0][out_key]
     q = torch.empty((T, w.n_h, w.D), device=dev, dtype=torch.bfloat16)
+    qa = torch.empty((T, w.n_h, w.d_h + w.d_r), device=dev, dtype=torch.bfloat16) if args.order_a else None
     o_lat = torch.empty((T, w.n_h, w.d_c), device=dev, dtype=torch.bfloat16)
     lse = torch.empty((T, w.n_h), device=dev, dtype=torch.float32)
     ws = {op: torch.empty(max(1, mla.workspace_size(p, op, w.B if op == mla.OP_DECODE else T, w.n_q)),
                           dtype=torch.uint8, device=dev)
           for op in (mla.OP_APPEND, mla.OP_ABSORB, mla.OP_DECODE, mla.OP_OUT_PROJ, mla.OP_O_PROJ,
                      mla.OP_O_PROJ_LATENT, mla.OP_ABSORB_MERGED, mla.OP_FRONT_END)}
+    if args.order_a:
+        ws[mla.OP_QUERY_HEADS] = torch.empty(max(1, mla.workspace_size(p, mla.OP_QUERY_HEADS, T)), dtype=torch.uint8,
+                                             device=dev)
+        ws[mla.OP_ATTEND_A] = torch.empty(max(1, mla.workspace_size(p, mla.OP_ATTEND_A, w.B, w.n_q,
+                                                                    mla.cache_rows(caches[0]))),
+                                          dtype=torch.uint8, device=dev)
     ws[mla.OP_DECODE] = torch.empty(max(1, mla.workspace_size(p, mla.OP_DECODE, w.B, w.n_q, mla.cache_capacity(caches[0]),
                                                               args.num_splits)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)  # graph capture needs a non-default stream
@@ -275,6 +289,22 @@ def run_ours(args, rank, world, local_rank):
     def step(i=None, b=0, c=None):
         x_ = bufs[b]
         cache = caches[(i if c is None else c) % n_copies if (i is not None or c is not None) else 0]
+        if args.order_a:
+            ev_fork.record(stream)
+            side.wait_event(ev_fork)
+            mla.mla_cache_append(p, x_["h"], W["W_DKV"], W["W_KR"], x_["sidx"], x_["pos"], cache,
+                                 ws=ws[mla.OP_APPEND], stream=side)
+            ev_join.record(side)
+            mla.mla_query_heads(p, x_["h"], W["W_DQ"], W["W_UQ"], W["W_QR"], x_["pos"], qa, ws=ws[mla.OP_QUERY_HEADS],
+                                stream=stream)
+            stream.wait_event(ev_join)
+            if i is not None:
+                ev_dec[i][0].record(stream)
+            mla.mla_attend_order_a(p, qa, W["W_UK"], W["W_UV"], cache, x_["sl"], w.n_q, x_["o"].view(T, w.n_h, w.d_h),
+                                   ws=ws[mla.OP_ATTEND_A], stream=stream)
+            if i is not None:
+                ev_dec[i][1].record(stream)
+            return
         if args.fused_front_end:
             mla.mla_front_end(p, x_["h"], W["W_DKV"], W["W_KR"], W["W_DQ"], W["W_UQ"], W["W_QR"], W["W_UK"],
                               x_["sidx"], x_["pos"], cache, q, ws=ws[mla.OP_FRONT_END], stream=stream)
@@ -565,6 +595,37 @@ def config_of(w, n, x, n_copies=None, args=None):
             "step": step_text(args)}
 
 
+def order_a_line(args, r, w, x, work, peaks, peak_kind, world):
+    """Bench line of the order-A step. Its dominant call, mla_attend_order_a,
+    is a dense contraction: the attention (n_h heads, 2 (d_h + d_r) + 2 d_h flops
+    per query row and visible key) and the decompression of K_C and V for every
+    physical cache row (2 x 2 d_h d_c flops per head and row); roofline = those
+    flops at the measured bf16 tensor peak."""
+    rows = int(np.prod(x.cache.shape[:2]))
+    attn = 2 * w.n_h * work["tokens_attended"] * (w.d_h + w.d_r + w.d_h)
+    decomp = 2 * 2 * w.n_h * w.d_h * w.d_c * rows
+    flops = attn + decomp
+    dec_s = r["dec_ms"] * 1e-3
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    return {
+        "metric": METRIC, "value": r["step_ms"] * 1e3, "unit": "µs/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**config_of(w, world, x, r["n_copies"], args),
+                   "step": "append + per-head queries + order-A attention (decompress K/V, then 192-d attention)"},
+        "attend_order_a_us": r["dec_ms"] * 1e3, "attend_us_p10_p50_p90": r["dec_pct"],
+        "roofline": {"kernel": "mla_attend_order_a (decompression GEMMs + k_attend_a)", "bound": "tensor",
+                     "achieved": flops / dec_s / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": t_tc / dec_s, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_flops": flops, "attention_flops": attn, "decompression_flops": decomp,
+                     "roofline_us": t_tc * 1e6},
+        "e2e": {"value": r["e2e_ms"] * 1e3, "unit": "µs/step", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"], "clocks": r["clocks"],
+        "launch": "the step's C-ABI calls captured once into a CUDA graph, replayed",
+    }
+
+
 def o_proj_line(w, op_ms, peaks, absorbed):
     """Timing of the output projection against its weight-streaming roofline:
     W_O (d x n_h d_h) or, absorbed, W_OV (d x n_h d_c), bf16."""
@@ -603,6 +664,9 @@ def main():
     w, x = r["w"], r["x"]
     work = synth.algorithmic_work(w, x.seq_lens)
     peaks, peak_kind = load_peaks()
+    if args.order_a:
+        print(json.dumps(order_a_line(args, r, w, x, work, peaks, peak_kind, world)))
+        return
     us = r["step_ms"] * 1e3
     dec_s = r["dec_ms"] * 1e-3
     cache_gbs = work["cache_bytes"] / dec_s / 1e9

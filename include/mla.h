@@ -225,6 +225,32 @@ mla_status mla_front_end(const mla_dims *dims, const void *h, const void *W_DKV,
                          const int32_t *seq_idx, const int32_t *positions, int32_t T, const mla_cache *cache,
                          void *q, void *ws, size_t ws_bytes, void *stream);
 
+/* Per-head queries without absorption, for order A (MLA walk-through,
+ * section 1 step 3): c_Q = W_DQ h_t; q_C,h = W_UQ_h c_Q (d_h);
+ * q_R,h = RoPE(W_QR_h c_Q, positions[t]) (d_r), written as
+ *   qa (output) [T][n_h][d_h + d_r] = [q_C,h | q_R,h], storage dtype
+ * (c_Q rounded once to the storage dtype, as in mla_absorb_q). */
+mla_status mla_query_heads(const mla_dims *dims, const void *h, const void *W_DQ, const void *W_UQ,
+                           const void *W_QR, const int32_t *positions, int32_t T, void *qa, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/* Attention in order A, the training form (MLA walk-through, section 3 order
+ * A: decompress, then the ordinary dot product): for head h and cached row i
+ *   K_h,i = [W_UK_h c_KV_i ; k_R,i] (d_h + d_r),  V_h,i = W_UV_h c_KV_i (d_h),
+ * and for token row t = b*n_q + j (new token j of sequence b at position
+ * L_b - n_q + j, causal within the chunk of n_q tokens; L_b = seq_lens[b]):
+ *   o[t][h] = sum_i softmax_i(scale qa[t][h] . K_h,i) V_h,i,  i <= L_b - n_q + j,
+ * the same o as mla_decode followed by mla_out_proj (order B), up to rounding.
+ *   qa [B*n_q][n_h][d_h + d_r] (mla_query_heads)   W_UK, W_UV [n_h*d_h][d_c]
+ *   o (output) [B*n_q][n_h][d_h], storage dtype.
+ * The tensor-core path decompresses K_C and V for every physical cache row
+ * into the workspace (bf16, 2 * n_h * rows * d_h * 2 bytes; rows =
+ * num_blocks * block_size, or num_seqs * max_len) and stores o rounded once.
+ * Bad seq_lens raise MLA_ERR_DEVICE_DATA and leave that sequence unwritten. */
+mla_status mla_attend_order_a(const mla_dims *dims, const void *qa, const void *W_UK, const void *W_UV,
+                              const mla_cache *cache, const int32_t *seq_lens, int32_t B, int32_t n_q, void *o,
+                              void *ws, size_t ws_bytes, void *stream);
+
 /* Self-test of the failure path (no counterpart on the pages). Launches one
  * small projection kernel whose copy engine is told to issue nothing, so that
  * its MMA thread's bounded wait runs out after wait_ns nanoseconds; the kernel
@@ -239,10 +265,13 @@ mla_status mla_selftest_timeout(uint64_t wait_ns, void *scratch, size_t scratch_
  * num_splits are used by decode only. max_seq_len bounds the tiles of a row
  * for forced splits (0 = unknown: the size then covers num_splits pieces for
  * every row); mla_decode itself requires the size for max_seq_len = the
- * cache's capacity (max_len, or max_blocks_per_seq * block_size). */
+ * cache's capacity (max_len, or max_blocks_per_seq * block_size). For
+ * MLA_OP_ATTEND_A, max_seq_len is the number of physical cache rows
+ * (num_blocks * block_size, or num_seqs * max_len). */
 enum {
   MLA_OP_APPEND = 0, MLA_OP_ABSORB = 1, MLA_OP_DECODE = 2, MLA_OP_OUT_PROJ = 3, MLA_OP_O_PROJ = 4,
-  MLA_OP_O_PROJ_LATENT = 5, MLA_OP_ABSORB_MERGED = 6, MLA_OP_FRONT_END = 7, MLA_OP_ABSORB_WO = 8
+  MLA_OP_O_PROJ_LATENT = 5, MLA_OP_ABSORB_MERGED = 6, MLA_OP_FRONT_END = 7, MLA_OP_ABSORB_WO = 8,
+  MLA_OP_QUERY_HEADS = 9, MLA_OP_ATTEND_A = 10
 };
 size_t mla_workspace_size(const mla_dims *dims, int32_t op, int32_t rows, int32_t n_q,
                           int64_t max_seq_len, int32_t num_splits);

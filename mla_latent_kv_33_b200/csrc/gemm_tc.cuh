@@ -27,6 +27,7 @@ enum Epi : int {
   EPI_BF16 = 1,     // bf16 dst[batch * e_bs + n * e_ns + m]
   EPI_UQ = 2,       // rows < e_split: bf16 q_C at dst[n * e_split + m]; rows above: q_R rotated
                     // by RoPE at positions[n], stored at q[n][h][d_c + i] (m - e_split = h * d_r + i)
+  EPI_QA = 3,       // as EPI_UQ, but q_C row m = h * d_c + i goes to q[n][h][i] (d_c = the q_C width)
 };
 
 struct Params {
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     const int m = m0 + row;
     const int n_base = n_tile * p.n_tile;
     float *out = p.out + (static_cast<int64_t>(batch) * p.splits + split) * p.n_total * p.m_total;
-    const bool rope_tile = p.epi == EPI_UQ && m0 >= p.e_split;  // whole M tiles are q_C or q_R
+    const bool rope_tile = (p.epi == EPI_UQ || p.epi == EPI_QA) && m0 >= p.e_split;  // whole M tiles are q_C or q_R
     for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
       uint32_t v[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * sp) << 16) + c0, v);
@@ -217,11 +218,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
           }
         }
       } else if (!rope_tile) {
+        const int64_t qrow = static_cast<int64_t>(p.n_h) * (p.d_c + p.d_r);
+        const int64_t qa_off = static_cast<int64_t>(m / max(p.d_c, 1)) * (p.d_c + p.d_r) + m % max(p.d_c, 1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int n = n_base + c0 + c;
-          if (c0 + c < p.n_tile && n < p.n_total)
-            p.dst[static_cast<int64_t>(n) * p.e_split + m] = __float2bfloat16_rn(__uint_as_float(v[c]));
+          if (c0 + c < p.n_tile && n < p.n_total) {
+            const __nv_bfloat16 x = __float2bfloat16_rn(__uint_as_float(v[c]));
+            if (p.epi == EPI_QA) p.q[n * qrow + qa_off] = x;
+            else p.dst[static_cast<int64_t>(n) * p.e_split + m] = x;
+          }
         }
       } else {
         // q_R rows: lanes (2k, 2k+1) hold the RoPE pair (x[2i], x[2i+1]); the

@@ -27,6 +27,7 @@
 #include "simt.cuh"
 #include "gemm_tc.cuh"
 #include "decode_tc.cuh"
+#include "prefill_tc.cuh"
 
 namespace {
 
@@ -86,7 +87,7 @@ mla_status launched(cudaError_t e, const char *what) {
 
 // cudaFuncSetAttribute applies to the current device: a kernel's dynamic
 // shared memory limit is raised once per device (bit `device` of its mask).
-enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_KERNELS = 3 };
+enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_ATTEND_A = 3, SMEM_KERNELS = 4 };
 std::atomic<uint64_t> g_smem_raised[SMEM_KERNELS];
 
 mla_status raise_smem_limit(const void *kernel, SmemKernel which, int bytes, const char *what) {
@@ -148,6 +149,11 @@ mla::CacheView view_of(const mla_cache *c) {
   v.max_blocks_per_seq = c->max_blocks_per_seq;
   v.num_seqs = c->num_seqs;
   return v;
+}
+
+// Longest sequence the cache can hold (bounds the tiles of a row).
+int64_t cache_capacity(const mla_cache *c) {
+  return c->paged ? static_cast<int64_t>(c->max_blocks_per_seq) * c->block_size : c->max_len;
 }
 
 bool tc_geometry(const mla_dims *d) {
@@ -342,6 +348,40 @@ mla_status simt_o_proj_latent(const mla_dims *d, const void *o_lat, const void *
   return cuda_check("o_proj (absorbed, CUDA cores)");
 }
 
+
+template <typename T>
+mla_status simt_query_heads(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                            const int32_t *positions, int Tn, void *qa, void *ws, cudaStream_t st) {
+  const int64_t HD = static_cast<int64_t>(d->n_h) * d->d_h;
+  const int64_t HR = static_cast<int64_t>(d->n_h) * d->d_r;
+  float *cq = static_cast<float *>(ws);                  // [T][d_cq]
+  float *qc = cq + static_cast<int64_t>(Tn) * d->d_cq;  // [T][n_h][d_h]
+  float *qr = qc + Tn * HD;                              // [T][n_h][d_r]
+  launch_linear<T>(static_cast<const T *>(W_DQ), 0, d->d, 1, h, false, 0, d->d, cq, 0, d->d_cq, d->d_cq, d->d, Tn, 1,
+                   st);
+  launch_linear<T>(static_cast<const T *>(W_UQ), 0, d->d_cq, 1, cq, true, 0, d->d_cq, qc, 0, HD, static_cast<int>(HD),
+                   d->d_cq, Tn, 1, st);
+  launch_linear<T>(static_cast<const T *>(W_QR), 0, d->d_cq, 1, cq, true, 0, d->d_cq, qr, 0, HR, static_cast<int>(HR),
+                   d->d_cq, Tn, 1, st);
+  // qa[t][h] = [q_C (d_h) | RoPE(q_R) (d_r)]: the q store with d_h in place of d_c
+  MLA_LAUNCH(mla::k_simt_q_store<T><<<Tn * d->n_h, 128, 0, st>>>(qc, qr, d->n_h, d->d_h, d->d_r, d->rope_base,
+                                                                    positions, static_cast<T *>(qa)));
+  return cuda_check("query heads (CUDA cores)");
+}
+
+size_t simt_query_heads_ws(const mla_dims *d, int Tn) {
+  return sizeof(float) * static_cast<size_t>(Tn) * (d->d_cq + static_cast<size_t>(d->n_h) * (d->d_h + d->d_r));
+}
+
+template <typename T>
+mla_status simt_attend_a(const mla_dims *d, const void *qa, const void *W_UK, const void *W_UV, const mla_cache *c,
+                         const int32_t *seq_lens, int B, int n_q, void *o, cudaStream_t st) {
+  const int rows = B * n_q * d->n_h;
+  MLA_LAUNCH(mla::k_simt_attend_a<T><<<rows, 128, 2 * 128 * sizeof(float), st>>>(
+      static_cast<const T *>(qa), static_cast<const T *>(W_UK), static_cast<const T *>(W_UV), view_of(c), seq_lens,
+      n_q, d->n_h, d->d_h, d->d_c, d->d_r, softmax_scale(d), static_cast<T *>(o)));
+  return cuda_check("order-A attention (CUDA cores)");
+}
 
 // ------------------------------------------------------------- TMA maps --
 
@@ -799,6 +839,127 @@ mla_status tc_o_proj_latent(const mla_dims *d, const void *o_lat, const void *W_
                   "o_proj (absorbed) finalize");
 }
 
+// ---- order A: query heads without absorption, decompression, 192-d attention ----
+size_t tc_query_heads_ws(const mla_dims *d, int T) {
+  const GemmShape cq = gemm_shape(d->d_cq, T, d->d, 1, true);
+  return align256(gemm_part_bytes(cq, T)) + static_cast<size_t>(T) * d->d_cq * 2;
+}
+
+mla_status tc_query_heads(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                          const int32_t *positions, int T, void *qa, void *ws, cudaStream_t st) {
+  const size_t cq_off = align256(gemm_part_bytes(gemm_shape(d->d_cq, T, d->d, 1, true), T));
+  mla_status s = tc_query_latent(d, h, W_DQ, T, ws, cq_off, st);
+  if (s != MLA_OK) return s;
+  const __nv_bfloat16 *cq = reinterpret_cast<const __nv_bfloat16 *>(static_cast<uint8_t *>(ws) + cq_off);
+  const int HD = d->n_h * d->d_h;
+  // [q_C ; q_R] = [W_UQ ; W_QR] c_Q: q_C,h into qa[t][h][0, d_h), q_R,h rotated into qa[t][h][d_h, d_h + d_r)
+  const GemmShape g = gemm_shape(d->n_h * (d->d_h + d->d_r), T, d->d_cq, 1, false);
+  CUtensorMap ta, ta2, tb;
+  if ((s = make_tmap_bf16(&ta, W_UQ, d->d_cq, HD, d->d_cq * 2ull, 64, 128, "W_UQ")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&ta2, W_QR, d->d_cq, d->n_h * d->d_r, d->d_cq * 2ull, 64, 128, "W_QR")) != MLA_OK) return s;
+  if ((s = make_tmap_bf16(&tb, cq, d->d_cq, T, d->d_cq * 2ull, 64, g.n_tile, "c_Q")) != MLA_OK) return s;
+  G::Params p{};
+  p.epi = G::EPI_QA;
+  p.e_split = HD;
+  p.q = static_cast<__nv_bfloat16 *>(qa);
+  p.n_h = d->n_h;
+  p.d_c = d->d_h;  // the q_C width of a qa row; q_R follows it
+  p.d_r = d->d_r;
+  p.rope_base = d->rope_base;
+  p.positions = positions;
+  GemmOperands op = operands(ta, tb);
+  op.a2 = &ta2;
+  op.m_split = HD;
+  return launch_gemm(op, g, T, p, st);
+}
+
+int64_t cache_rows_of(const mla_cache *c) {
+  return c->paged ? c->num_blocks * c->block_size : static_cast<int64_t>(c->num_seqs) * c->max_len;
+}
+
+// decompressed K_C and V: [n_h][rows][d_h] bf16 each
+size_t tc_attend_a_ws(const mla_dims *d, int64_t rows) {
+  return 2 * align256(static_cast<size_t>(d->n_h) * rows * d->d_h * 2);
+}
+
+mla_status tc_attend_a(const mla_dims *d, const void *qa, const void *W_UK, const void *W_UV, const mla_cache *c,
+                       const int32_t *seq_lens, int B, int n_q, void *o, void *ws, cudaStream_t st) {
+  namespace P = mla::pre;
+  const int64_t R = cache_rows_of(c);
+  if (c->paged && c->block_size % P::BLK != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "order-A attention needs block_size to be a multiple of %d", P::BLK);
+  if (R >= 0x7fff0000LL || (R + 255) / 256 > 65535)
+    return fail(MLA_ERR_UNSUPPORTED, "order-A attention: too many cache rows");
+  const int HD = d->n_h * d->d_h;
+  const int64_t D = d->d_c + d->d_r;
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(w8);
+  __nv_bfloat16 *vv = reinterpret_cast<__nv_bfloat16 *>(w8 + align256(static_cast<size_t>(d->n_h) * R * d->d_h * 2));
+  mla_status s;
+  // decompression over every physical cache row: X_h[r][i] = sum_j W[h d_h + i][j] c_KV[r][j]
+  const GemmShape g = gemm_shape(d->d_h, static_cast<int>(R), d->d_c, d->n_h, false);
+  CUtensorMap tb;
+  if ((s = make_tmap_bf16(&tb, c->data, d->d_c, R, D * 2, 64, g.n_tile, "cache (c_KV)")) != MLA_OK) return s;
+  const void *Ws[2] = {W_UK, W_UV};
+  __nv_bfloat16 *dsts[2] = {kc, vv};
+  for (int u = 0; u < 2; ++u) {
+    CUtensorMap ta;
+    if ((s = make_tmap_bf16(&ta, Ws[u], d->d_c, HD, d->d_c * 2ull, 64, 128, u == 0 ? "W_UK" : "W_UV")) != MLA_OK)
+      return s;
+    G::Params p{};
+    p.epi = G::EPI_BF16;
+    p.dst = dsts[u];
+    p.e_bs = R * d->d_h;
+    p.e_ns = d->d_h;
+    GemmOperands op = operands(ta, tb);
+    op.a_batch_rows = d->d_h;
+    if ((s = launch_gemm(op, g, static_cast<int>(R), p, st)) != MLA_OK) return s;
+  }
+  // attention
+  const int T = B * n_q;
+  CUtensorMap tm_q, tm_kc, tm_kr, tm_v;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(P::DQK), static_cast<uint64_t>(d->n_h), static_cast<uint64_t>(T)};
+    const uint64_t str[2] = {P::DQK * 2ull, static_cast<uint64_t>(d->n_h) * P::DQK * 2};
+    const uint32_t box[3] = {64, 1, P::QROWS};
+    if ((s = make_tmap_nd(&tm_q, qa, 3, dims, str, box, "qa")) != MLA_OK) return s;
+  }
+  for (int u = 0; u < 2; ++u) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d->d_h), static_cast<uint64_t>(R), static_cast<uint64_t>(d->n_h)};
+    const uint64_t str[2] = {d->d_h * 2ull, static_cast<uint64_t>(R) * d->d_h * 2};
+    const uint32_t box[3] = {64, P::BLK, 1};
+    if ((s = make_tmap_nd(u == 0 ? &tm_kc : &tm_v, dsts[u], 3, dims, str, box, u == 0 ? "K_C" : "V")) != MLA_OK)
+      return s;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(R)}, str[1] = {static_cast<uint64_t>(D) * 2};
+    const uint32_t box[2] = {64, P::BLK};
+    if ((s = make_tmap_nd(&tm_kr, c->data, 2, dims, str, box, "cache (k_R)")) != MLA_OK) return s;
+  }
+  P::Params pp{};
+  pp.seq_lens = seq_lens;
+  pp.block_table = c->block_table;
+  pp.max_len = c->max_len;
+  pp.rows = R;
+  pp.paged = c->paged;
+  pp.block_size = c->block_size;
+  pp.max_blocks_per_seq = c->max_blocks_per_seq;
+  pp.num_blocks_i32 = static_cast<int32_t>(c->paged ? c->num_blocks : 0);
+  pp.B = B;
+  pp.n_q = n_q;
+  pp.n_h = d->n_h;
+  pp.qblocks = (n_q + P::QROWS - 1) / P::QROWS;
+  pp.capacity = cache_capacity(c);
+  pp.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
+  pp.o = static_cast<__nv_bfloat16 *>(o);
+  if ((s = raise_smem_limit(reinterpret_cast<const void *>(P::k_attend_a), SMEM_ATTEND_A, P::SMEM_BYTES,
+                            "order-A attention: set shared memory size")) != MLA_OK)
+    return s;
+  return launched(launch_tc(P::k_attend_a, dim3(d->n_h * B * pp.qblocks), dim3(P::NUM_THREADS), P::SMEM_BYTES, st,
+                            tm_q, tm_kc, tm_kr, tm_v, pp),
+                  "order-A attention (tensor cores)");
+}
+
 // ---- failure-path self-test: a projection GEMM whose producer issues nothing ----
 // The MMA thread's first wait runs out after wait_ns; the kernel records the
 // timeout in the device error word and unwinds (no copy is in flight; tensor
@@ -910,11 +1071,6 @@ int decode_clusters(int sms) {
   n = std::max(1, std::min(n, sms / 2));
   if (dev >= 0 && dev < MAX_DEVICES) g_decode_clusters[dev].store(n, std::memory_order_release);
   return n;
-}
-
-// Longest sequence the cache can hold (bounds the tiles of a row).
-int64_t cache_capacity(const mla_cache *c) {
-  return c->paged ? static_cast<int64_t>(c->max_blocks_per_seq) * c->block_size : c->max_len;
 }
 
 mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const int32_t *seq_lens, int B, int n_q,
@@ -1087,7 +1243,7 @@ int32_t mla_get_launch_overlap(void) { return g_overlap.load(std::memory_order_r
 
 int32_t mla_uses_tensor_cores(const mla_dims *d, int32_t op) {
   if (d == nullptr || !tc_geometry(d)) return 0;
-  return (op >= MLA_OP_APPEND && op <= MLA_OP_ABSORB_WO) ? 1 : 0;
+  return (op >= MLA_OP_APPEND && op <= MLA_OP_ATTEND_A) ? 1 : 0;
 }
 
 size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n_q, int64_t max_seq_len,
@@ -1105,6 +1261,8 @@ size_t mla_workspace_size(const mla_dims *d, int32_t op, int32_t rows, int32_t n
     case MLA_OP_ABSORB_MERGED: return tc ? tc_absorb_merged_ws(d, rows) : simt_absorb_merged_ws(d, rows);
     case MLA_OP_FRONT_END:
       return tc ? tc_front_ws(d, rows) : std::max(simt_append_ws(d, rows), simt_absorb_ws(d, rows));
+    case MLA_OP_QUERY_HEADS: return tc ? tc_query_heads_ws(d, rows) : simt_query_heads_ws(d, rows);
+    case MLA_OP_ATTEND_A: return tc && max_seq_len > 0 ? tc_attend_a_ws(d, max_seq_len) : 0;
   }
   return 0;
 }
@@ -1314,6 +1472,44 @@ mla_status mla_front_end(const mla_dims *d, const void *h, const void *W_DKV, co
   // CUDA-core dims: the two calls one after the other (each reads h)
   if ((s = mla_cache_append(d, h, W_DKV, W_KR, seq_idx, positions, T, c, ws, ws_bytes, stream)) != MLA_OK) return s;
   return mla_absorb_q(d, h, W_DQ, W_UQ, W_QR, W_UK, positions, T, q, ws, ws_bytes, stream);
+}
+
+mla_status mla_query_heads(const mla_dims *d, const void *h, const void *W_DQ, const void *W_UQ, const void *W_QR,
+                           const int32_t *positions, int32_t T, void *qa, void *ws, size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (T <= 0) return fail(MLA_ERR_INVALID_ARG, "T must be positive");
+  if (!h || !W_DQ || !W_UQ || !W_QR || !positions || !qa)
+    return fail(MLA_ERR_INVALID_ARG, "query_heads: NULL tensor argument");
+  if (!aligned16(h) || !aligned16(W_DQ) || !aligned16(W_UQ) || !aligned16(W_QR) || !aligned16(qa))
+    return fail(MLA_ERR_INVALID_ARG, "query_heads: tensors must be 16-byte aligned");
+  const size_t need = mla_workspace_size(d, MLA_OP_QUERY_HEADS, T, 1, 0, 0);
+  if (ws_bytes < need || (need && !ws)) return fail(MLA_ERR_WORKSPACE, "query_heads needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_query_heads(d, h, W_DQ, W_UQ, W_QR, positions, T, qa, ws, st);
+  if (d->dtype == MLA_BF16) return simt_query_heads<__nv_bfloat16>(d, h, W_DQ, W_UQ, W_QR, positions, T, qa, ws, st);
+  return simt_query_heads<float>(d, h, W_DQ, W_UQ, W_QR, positions, T, qa, ws, st);
+}
+
+mla_status mla_attend_order_a(const mla_dims *d, const void *qa, const void *W_UK, const void *W_UV,
+                              const mla_cache *c, const int32_t *seq_lens, int32_t B, int32_t n_q, void *o, void *ws,
+                              size_t ws_bytes, void *stream) {
+  mla_status s = check_dims(d);
+  if (s != MLA_OK) return s;
+  if (B <= 0 || n_q <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_q must be positive");
+  if (!qa || !W_UK || !W_UV || !seq_lens || !o) return fail(MLA_ERR_INVALID_ARG, "attend_order_a: NULL tensor argument");
+  if (!aligned16(qa) || !aligned16(W_UK) || !aligned16(W_UV) || !aligned16(o))
+    return fail(MLA_ERR_INVALID_ARG, "attend_order_a: tensors must be 16-byte aligned");
+  if ((s = check_cache(c, d->d_c + d->d_r)) != MLA_OK) return s;
+  if (B > c->num_seqs) return fail(MLA_ERR_INVALID_ARG, "B exceeds cache->num_seqs");
+  if (d->d_h > 128 || d->d_r > 128) return fail(MLA_ERR_UNSUPPORTED, "attend_order_a: d_h and d_r must be <= 128");
+  const size_t need = mla_workspace_size(d, MLA_OP_ATTEND_A, B, n_q, cache_rows_of(c), 0);
+  if (ws_bytes < need || (need && !ws))
+    return fail(MLA_ERR_WORKSPACE, "attend_order_a needs %zu workspace bytes", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_geometry(d)) return tc_attend_a(d, qa, W_UK, W_UV, c, seq_lens, B, n_q, o, ws, st);
+  if (d->dtype == MLA_BF16) return simt_attend_a<__nv_bfloat16>(d, qa, W_UK, W_UV, c, seq_lens, B, n_q, o, st);
+  return simt_attend_a<float>(d, qa, W_UK, W_UV, c, seq_lens, B, n_q, o, st);
 }
 
 mla_status mla_selftest_timeout(uint64_t wait_ns, void *scratch, size_t scratch_bytes, void *stream) {

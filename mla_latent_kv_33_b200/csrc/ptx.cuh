@@ -161,6 +161,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
       : "memory");
 }
 
+// 3-D tiled load into this CTA's shared memory, completing on a barrier of
+// this CTA.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
 // 2-D tiled load into this CTA's shared memory whose completion is signalled
 // on a barrier that may live in the peer CTA of the pair (shared::cluster
 // address). No multicast: each CTA fetches its own tile.

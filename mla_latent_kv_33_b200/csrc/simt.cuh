@@ -96,6 +96,64 @@ __global__ void k_simt_q_store(const float *__restrict__ q_lat, const float *__r
   }
 }
 
+// Order A for one (token row t, head h) per block (d_h <= blockDim.x): for
+// every visible cached row i, thread k forms k_C,i[k] = W_UK_h[k] . c_KV_i and
+// v_i[k] = W_UV_h[k] . c_KV_i; the score is scale ([q_C ; q_R] . [k_C,i ; k_R,i])
+// and an online softmax accumulates o[k] = sum_i p_i v_i[k] / sum_i p_i.
+// qa [T][n_h][d_h + d_r], o [T][n_h][d_h]. Shared memory: 2 * blockDim floats.
+template <typename T>
+__global__ void k_simt_attend_a(const T *__restrict__ qa, const T *__restrict__ W_UK, const T *__restrict__ W_UV,
+                                CacheView cache, const int32_t *__restrict__ seq_lens, int n_q, int n_h, int d_h,
+                                int d_c, int d_r, float scale, T *__restrict__ o) {
+  extern __shared__ float red[];
+  const int t = blockIdx.x / n_h, h = blockIdx.x % n_h;
+  const int b = t / n_q, j = t % n_q;
+  const int L = seq_lens[b];
+  const int D = d_c + d_r, k = threadIdx.x;
+  if (L < n_q || (!cache.paged && L > cache.max_len) ||
+      (cache.paged && static_cast<int64_t>(L) > static_cast<int64_t>(cache.max_blocks_per_seq) * cache.block_size)) {
+    if (threadIdx.x == 0 && j == 0 && h == 0) dev_error(MLA_DEVERR_DATA);
+    return;
+  }
+  const int vis = L - n_q + 1 + j;
+  const T *q = qa + (static_cast<int64_t>(t) * n_h + h) * (d_h + d_r);
+  const T *wk = W_UK + static_cast<int64_t>(h) * d_h * d_c + static_cast<int64_t>(k) * d_c;
+  const T *wv = W_UV + static_cast<int64_t>(h) * d_h * d_c + static_cast<int64_t>(k) * d_c;
+  const T *data = static_cast<const T *>(cache.data);
+  float m = -INFINITY, l = 0.f, acc = 0.f;
+  for (int i = 0; i < vis; ++i) {
+    const int64_t row = cache_row(cache, b, i);
+    if (row < 0) {
+      if (threadIdx.x == 0) dev_error(MLA_DEVERR_DATA);
+      return;
+    }
+    const T *c = data + row * D;
+    float kc = 0.f, vv = 0.f;
+    if (k < d_h)
+      for (int e = 0; e < d_c; ++e) {
+        const float x = ld_f(c + e);
+        kc += ld_f(wk + e) * x;
+        vv += ld_f(wv + e) * x;
+      }
+    float part = k < d_h ? ld_f(q + k) * kc : 0.f;
+    if (k < d_r) part += ld_f(q + d_h + k) * ld_f(c + d_c + k);
+    red[k] = part;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (k < w) red[k] += red[k + w];
+      __syncthreads();
+    }
+    const float s = scale * red[0];
+    __syncthreads();
+    const float mn = fmaxf(m, s);
+    const float a = __expf(m - mn), pw = __expf(s - mn);  // m = -inf on the first row: a = 0
+    l = l * a + pw;
+    acc = acc * a + pw * vv;
+    m = mn;
+  }
+  if (k < d_h) o[(static_cast<int64_t>(t) * n_h + h) * d_h + k] = from_f<T>(acc / l);
+}
+
 template <typename T>
 __global__ void k_simt_store(const float *__restrict__ src, T *__restrict__ dst, int64_t n) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;

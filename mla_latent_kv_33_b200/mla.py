@@ -24,7 +24,7 @@ MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUD
     MLA_ERR_DEVICE_DATA = range(7)
 MLA_BF16, MLA_FP32 = 0, 1
 OP_APPEND, OP_ABSORB, OP_DECODE, OP_OUT_PROJ, OP_O_PROJ, OP_O_PROJ_LATENT, OP_ABSORB_MERGED, OP_FRONT_END, \
-    OP_ABSORB_WO = range(9)
+    OP_ABSORB_WO, OP_QUERY_HEADS, OP_ATTEND_A = range(11)
 
 
 class Dims(C.Structure):
@@ -55,6 +55,9 @@ _lib.mla_absorb_q_merged.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, C.c_in
 _lib.mla_front_end.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_int32,
                                C.POINTER(CacheDesc), _P, _P, _S, _P]
 _lib.mla_selftest_timeout.argtypes = [C.c_uint64, _P, _S, _P]
+_lib.mla_query_heads.argtypes = [C.POINTER(Dims), _P, _P, _P, _P, _P, C.c_int32, _P, _P, _S, _P]
+_lib.mla_attend_order_a.argtypes = [C.POINTER(Dims), _P, _P, _P, C.POINTER(CacheDesc), _P, C.c_int32, C.c_int32, _P,
+                                    _P, _S, _P]
 _lib.mla_workspace_size.argtypes = [C.POINTER(Dims), C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_int32]
 _lib.mla_workspace_size.restype = C.c_size_t
 _lib.mla_get_device_error.argtypes = [_P]
@@ -66,7 +69,8 @@ _lib.mla_uses_tensor_cores.restype = C.c_int32
 _lib.mla_kernel_launches.restype = C.c_uint64
 for _f in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_decode_noalloc", "mla_out_proj", "mla_o_proj",
            "mla_get_device_error", "mla_set_launch_overlap", "mla_get_launch_overlap", "mla_absorb_wo",
-           "mla_o_proj_latent", "mla_absorb_merge", "mla_absorb_q_merged", "mla_front_end", "mla_selftest_timeout"):
+           "mla_o_proj_latent", "mla_absorb_merge", "mla_absorb_q_merged", "mla_front_end", "mla_selftest_timeout",
+           "mla_query_heads", "mla_attend_order_a"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -218,6 +222,26 @@ def mla_front_end(p: Dims, h, W_DKV, W_KR, W_DQ, W_UQ, W_QR, W_UK, seq_idx, posi
     _check(_lib.mla_front_end(C.byref(p), _ptr(h), _ptr(W_DKV), _ptr(W_KR), _ptr(W_DQ), _ptr(W_UQ), _ptr(W_QR),
                               _ptr(W_UK), _ptr(seq_idx), _ptr(positions), T, C.byref(cache.desc), _ptr(q), _ptr(ws),
                               nbytes, _stream(stream)), "mla_front_end")
+
+
+def cache_rows(cache: "Cache") -> int:
+    """Physical rows of the cache (the size mla_attend_order_a decompresses)."""
+    d = cache.desc
+    return d.num_blocks * d.block_size if d.paged else d.num_seqs * d.max_len
+
+
+def mla_query_heads(p: Dims, h, W_DQ, W_UQ, W_QR, positions, qa, ws=None, stream=None):
+    T = h.shape[0]
+    ws, nbytes = _ws(p, OP_QUERY_HEADS, T, 1, ws)
+    _check(_lib.mla_query_heads(C.byref(p), _ptr(h), _ptr(W_DQ), _ptr(W_UQ), _ptr(W_QR), _ptr(positions), T, _ptr(qa),
+                                _ptr(ws), nbytes, _stream(stream)), "mla_query_heads")
+
+
+def mla_attend_order_a(p: Dims, qa, W_UK, W_UV, cache: Cache, seq_lens, n_q, o, ws=None, stream=None):
+    B = seq_lens.shape[0]
+    ws, nbytes = _ws(p, OP_ATTEND_A, B, n_q, ws, cache_rows(cache))
+    _check(_lib.mla_attend_order_a(C.byref(p), _ptr(qa), _ptr(W_UK), _ptr(W_UV), C.byref(cache.desc), _ptr(seq_lens),
+                                   B, n_q, _ptr(o), _ptr(ws), nbytes, _stream(stream)), "mla_attend_order_a")
 
 
 def mla_selftest_timeout(wait_ns: int, scratch, stream=None):

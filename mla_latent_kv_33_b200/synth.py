@@ -98,6 +98,10 @@ WORKLOADS = {
         L_lo=256, L_hi=32768, paged=True,
         note="DeepSeek-V3 dims, batch 128, lognormal seq_lens (median 4096, sigma 0.5, "
              "clipped 256..32768), 2 query tokens per sequence"),
+    "v2_prefill_c512": Workload(
+        "v2_prefill_c512", 5, **V2, B=4, n_q=512, lens="fixed", L=4096, paged=True,
+        note="DeepSeek-V2 dims, chunked prefill: 4 sequences, a chunk of 512 new tokens each at positions "
+             "3584..4095 (causal within the chunk), paged cache (block 64); the order-A (training form) workload"),
 }
 
 

@@ -168,7 +168,7 @@ def test_tensor_core_geometry_switch(m):
     assert all(m._lib.mla_uses_tensor_cores(C.byref(d), op) == 1 for op in range(5))
     assert m._lib.mla_uses_tensor_cores(C.byref(v2(m, dtype="fp32")), m.OP_DECODE) == 0
     assert m._lib.mla_uses_tensor_cores(C.byref(v2(m, n_h=64)), m.OP_DECODE) == 0
-    assert m._lib.mla_uses_tensor_cores(C.byref(d), 9) == 0
+    assert m._lib.mla_uses_tensor_cores(C.byref(d), 99) == 0
 
 
 def test_python_binding_raises_with_status_and_message(m):
