@@ -72,6 +72,9 @@ def parse():
     ap.add_argument("--cpu-sample-s", type=float, default=15.0, help="target seconds of oracle work")
     ap.add_argument("--num-splits", type=int, default=0,
                     help="mla_decode num_splits: 0 = automatic plan, S > 0 = each token row in min(S, its tiles) pieces")
+    ap.add_argument("--breakdown", action="store_true",
+                    help="diagnostic: also time the front of the step (append + query chain) and its tail "
+                         "(W_UV readout) with event pairs in the timed graph; the extra nodes add to the step time")
     ap.add_argument("--with-o-proj", action="store_true",
                     help="add the output projection y = W_O o (mla_o_proj) to every step and time it on its own")
     ap.add_argument("--o-proj-absorbed", action="store_true",
@@ -280,6 +283,8 @@ def run_ours(args, rank, world, local_rank):
                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
     ev_op = [(torch.cuda.Event(enable_timing=True, external=True),
               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
+    ev_front = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
+    ev_tail = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
 
     # the cache append and the query absorption are independent: the append
     # runs on a side stream, joined before the decode reads the cache
@@ -288,6 +293,8 @@ def run_ours(args, rank, world, local_rank):
 
     def step(i=None, b=0, c=None):
         x_ = bufs[b]
+        if i is not None and args.breakdown:
+            ev_front[i].record(stream)
         cache = caches[(i if c is None else c) % n_copies if (i is not None or c is not None) else 0]
         if args.order_a:
             ev_fork.record(stream)
@@ -329,6 +336,8 @@ def run_ours(args, rank, world, local_rank):
             ev_dec[i][1].record(stream)
         if not args.o_proj_absorbed:
             mla.mla_out_proj(p, o_lat, W["W_UV"], x_["o"], ws=ws[mla.OP_OUT_PROJ], stream=stream)
+        if i is not None and args.breakdown:
+            ev_tail[i].record(stream)
         if args.with_o_proj:
             if i is not None:
                 ev_op[i][0].record(stream)
@@ -407,6 +416,11 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = float(np.mean(dec_list))
     dec_pct = percentiles_us(dec_list)
     op_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_op])) if args.with_o_proj else None
+    breakdown = None
+    if args.breakdown and not args.order_a:
+        breakdown = {"front_us": float(np.mean([f.elapsed_time(d[0]) for f, d in zip(ev_front, ev_dec)])) * 1e3,
+                     "decode_us": dec_ms * 1e3,
+                     "tail_us": float(np.mean([d[1].elapsed_time(t) for d, t in zip(ev_dec, ev_tail)])) * 1e3}
 
     # End to end through the public API: every step copies its inputs in from
     # pinned host memory and its output o back, inside the timed region. The
@@ -463,7 +477,7 @@ def run_ours(args, rank, world, local_rank):
     del graph_1, graph_k
     return {"step_ms": step_ms, "dec_ms": dec_ms, "dec_pct": dec_pct, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
             "launch_mode": ("eager" if args.eager else "cuda_graph") + ("" if args.no_overlap else "+overlap"),
-            "launches": launches, "clocks": clk.summary(), "x": x, "w": w, "op_ms": op_ms, "n_copies": n_copies,
+            "launches": launches, "clocks": clk.summary(), "x": x, "w": w, "op_ms": op_ms, "breakdown": breakdown, "n_copies": n_copies,
             "tc": mla.uses_tensor_cores(p, mla.OP_DECODE)}
 
 
@@ -701,6 +715,7 @@ def main():
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
         **({"o_proj": o_proj_line(w, r["op_ms"], peaks, args.o_proj_absorbed)} if r["op_ms"] is not None else {}),
+        **({"breakdown": r["breakdown"]} if r.get("breakdown") else {}),
         "tensor_core_decode": r["tc"],
         "clocks": r["clocks"],
     }

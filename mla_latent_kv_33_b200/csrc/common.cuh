@@ -54,16 +54,22 @@ __device__ __forceinline__ double rope_theta(int pair, int d_r, double base) {
 // 2^17 and beyond keep full accuracy); on that range the fast hardware sine
 // and cosine (__sincosf: absolute error below 2^-21.4 there) are far more
 // accurate than the bf16 results, and they keep the unrolled epilogues small.
-__device__ __forceinline__ void rope_rotate(float &x0, float &x1, int pos, double theta) {
+__device__ __forceinline__ void rope_cos_sin(int pos, double theta, float &c, float &s) {
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   const double a = static_cast<double>(pos) * theta;
   const double k = rint(a * (1.0 / kTwoPi));
-  float s, c;
   __sincosf(static_cast<float>(fma(-k, kTwoPi, a)), &s, &c);
+}
+__device__ __forceinline__ void rope_apply(float &x0, float &x1, float c, float s) {
   const float y0 = x0 * c - x1 * s;
   const float y1 = x0 * s + x1 * c;
   x0 = y0;
   x1 = y1;
+}
+__device__ __forceinline__ void rope_rotate(float &x0, float &x1, int pos, double theta) {
+  float c, s;
+  rope_cos_sin(pos, theta, c, s);
+  rope_apply(x0, x1, c, s);
 }
 
 __device__ __forceinline__ void rope_pair(float &x0, float &x1, int pair, int d_r, int pos, double base) {

@@ -31,10 +31,10 @@
 //    explicit whole-block L2 prefetch ahead of the score loads measured
 //    slower: it added DRAM reads without removing the score loads' misses.)
 //  * Loads: a TMA instruction occupies its issuing warp for ~0.3 us whatever
-//    the box size (the lanes of a warp issue in parallel), so three producer
-//    warps share the ring, big slot s belonging to warp s mod 3: every slot's
-//    uses are issued in order by one warp, whose lanes issue an item's boxes
-//    together.
+//    the box size (the lanes of a warp issue in parallel), so four producer
+//    warps share the ring, one per big slot: every slot's uses are issued in
+//    order by one warp, whose lanes issue an item's boxes together, and no
+//    slot waits behind another slot's issue.
 //  * P lives in tensor memory, written by the softmax over the scores it was
 //    made from, as the A operand of PV. A pair MMA with M = 128 reads a row's
 //    16-wide K group from both lane m and lane m + 64 (one copy per half of
@@ -42,8 +42,8 @@
 //    (held by lane m) with 8 of the second's (lane m + 64); the two lanes
 //    trade their halves through shared memory. The value item pairs blocks v
 //    and v + 2 at a fixed 16 KB distance, so that one B descriptor spans both.
-//  * Warp roles: warps 0-2 load, warp 3 of CTA 0 issues the MMAs of the pair,
-//    warps 4-7 of both CTAs run the online softmax (fp32, exp2, O rescaled
+//  * Warp roles: warps 0-2 and 8 load, warp 3 of CTA 0 issues the MMAs of the
+//    pair, warps 4-7 of both CTAs run the online softmax (fp32, exp2, O rescaled
 //    only when the running max grows by more than 2^8) and the epilogue.
 //  * Work: the visible 256-token tiles of all token rows are concatenated and
 //    cut into equal contiguous ranges, one per cluster (persistent grid). A
@@ -68,10 +68,11 @@ namespace dec {
 
 constexpr int D = 576, DC = 512, DR = 64, HEADS = 128, HPC = 64;
 constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CTA / per block
-// 8 warps = 2 per SM sub-partition, so each thread may hold up to 255 registers
-constexpr int NUM_PRODUCERS = 3, WARP_MMA = 3, WARP_SOFTMAX = 4;
-constexpr int NUM_THREADS = 32 * (WARP_SOFTMAX + 4);
-constexpr int NBIG = 4;              // 32 KB ring slots; big slot s belongs to producer warp s % 3
+// 9 warps: producers 0-2 and 8 (producer index 3), the MMA warp 3, and the
+// softmax warps 4-7 (warp w reaches tensor-memory lanes 32 (w % 4) .. + 31)
+constexpr int NUM_PRODUCERS = 4, WARP_MMA = 3, WARP_SOFTMAX = 4, WARP_PROD3 = 8;
+constexpr int NUM_THREADS = 32 * 9;
+constexpr int NBIG = 4;              // 32 KB ring slots; big slot s belongs to producer s
 constexpr int SMALL_OWNER = 1, Q_OWNER = 2;
 constexpr int CHUNK_Q = HPC * 128;   // 64 heads x 64 columns
 constexpr int ATOM = BLK * 128;      // 64 rows x 64 columns (one 128-byte-swizzle atom column)
@@ -87,8 +88,8 @@ constexpr int OFF_SMALL = OFF_BIG + NBIG * BIG;
 constexpr int OFF_XBUF = OFF_SMALL + SMALL;
 constexpr int OFF_MISC = OFF_XBUF + XBUF_BYTES;
 constexpr int BAR_Q_FULL = 0, BAR_Q_EMPTY = 1, BAR_BIG_FULL = 2, BAR_BIG_EMPTY = BAR_BIG_FULL + NBIG,
-              BAR_SMALL_FULL = BAR_BIG_EMPTY + NBIG, BAR_SMALL_EMPTY = BAR_SMALL_FULL + 1,
-              BAR_V_LANDED = BAR_SMALL_EMPTY + 1, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
+              BAR_SMALL_FULL = BAR_BIG_EMPTY + NBIG,
+              BAR_V_LANDED = BAR_SMALL_FULL + 1, BAR_ZERO_DONE = BAR_V_LANDED + 1, BAR_S_FULL = BAR_ZERO_DONE + 1,
               BAR_P_FULL = BAR_S_FULL + 2, BAR_O_FULL = BAR_P_FULL + 1,
               BAR_O_FREE = BAR_O_FULL + 1, BAR_EXIT = BAR_O_FREE + 1, NUM_BARS = BAR_EXIT + 1;
 constexpr int MISC_RED = 256;               // float red[2][128]
@@ -149,20 +150,22 @@ __device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out)
   return (vis + TILE - 1) / TILE;
 }
 
-// First cache row of the 64-row block at token `pos` of sequence b, or
-// p.cache_rows (out of range: the TMA load zero-fills) when the block lies
-// past `vis` or its block-table entry is invalid.
 // Cache rows of the four 64-token blocks of a 256-token tile (positions
 // t0 + 64 v), or cache_rows (an out-of-range TMA coordinate: zero fill) for
-// blocks past the visible length. The four block-table entries are loaded
-// before any of them is checked, so that their latencies overlap.
-__device__ __forceinline__ void tile_rows(const Params &p, int b, int64_t t0, int vis, int32_t r4[4]) {
-  int32_t blk[4];
+// blocks past the visible length or with an invalid block-table entry. Two
+// steps: tile_blocks() issues the four block-table loads, rows_of_blocks()
+// checks and converts their values. The producers issue the loads of tile
+// i + 2 while they convert those of tile i + 1, loaded a whole tile earlier,
+// so that the check (a branch on the loaded value) never waits for memory.
+__device__ __forceinline__ void tile_blocks(const Params &p, int b, int64_t t0, int vis, int32_t blk[4]) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
     const int64_t pos = t0 + BLK * v;
     blk[v] = p.paged && pos < vis ? p.block_table[static_cast<int64_t>(b) * p.max_blocks_per_seq + pos / p.block_size] : 0;
   }
+}
+__device__ __forceinline__ void rows_of_blocks(const Params &p, int b, int64_t t0, int vis, const int32_t blk[4],
+                                               int32_t r4[4]) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
     const int64_t pos = t0 + BLK * v;
@@ -346,7 +349,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       mbar_init(bar(BAR_BIG_EMPTY + s), 1);
     }
     mbar_init(bar(BAR_SMALL_FULL), 1);
-    mbar_init(bar(BAR_SMALL_EMPTY), 1);
     mbar_init(bar(BAR_V_LANDED), 1);
     mbar_init(bar(BAR_ZERO_DONE), 8);
     for (int b = 0; b < 2; ++b) mbar_init(bar(BAR_S_FULL + b), 1);
@@ -439,14 +441,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   it0.k = cluster;
   it0.S = S;
 
-  if (warp < NUM_PRODUCERS) {
+  if (warp < WARP_MMA || warp == WARP_PROD3) {
     // --------------------------------------------------------- ring producers
     // Every producer warp walks the same item sequence and issues the items
     // of the slots it owns, so that each slot's uses are issued in order by
     // one warp (a parity wait on the slot's empty barrier is exact only when
     // the waiter is at most one phase ahead). Lane 0 waits for the slot and
     // arms its full barrier, then lane l issues box l of the item.
-    const int w = warp;
+    const int w = warp < WARP_MMA ? warp : 3;  // producer index
     const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
     PieceIter it = it0;
     Piece pc;
@@ -467,11 +469,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         use = nsmall++;
       }
       if ((big ? slot % NUM_PRODUCERS : SMALL_OWNER) != w) return 0;
-      const int eb = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
+      // the small slot's use u is tile u's score item; it is free once S(u)
+      // has completed (S_FULL of buffer u & 1, phase u >> 1)
+      const int eb = big ? BAR_BIG_EMPTY + slot : BAR_S_FULL + ((use - 1) & 1);
+      const uint32_t epar = big ? (use - 1) & 1 : ((use - 1) >> 1) & 1;
       *fb = big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL;
       bool good = true;
       if (lane == 0) {
-        if (use > 0) good = mbar_wait(bar(eb), (use - 1) & 1, abort_flag);
+        if (use > 0) good = mbar_wait(bar(eb), epar, abort_flag);
         if (good && rank == 0) mbar_arrive_expect_tx(bar(*fb), 2 * bytes);
       }
       return __shfl_sync(0xffffffffu, good, 0) ? (big ? OFF_BIG + slot * BIG : OFF_SMALL) : -1;
@@ -508,9 +513,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     };
     while (ok && it.next(p, pc)) {
       const int b = pc.bj / p.n_q;
-      auto rows_of = [&](int ti, int32_t *r4) { tile_rows(p, b, static_cast<int64_t>(ti) * TILE, pc.vis, r4); };
-      int32_t cur[4], prev[4], nxt[4] = {0, 0, 0, 0};
-      rows_of(pc.t_begin, cur);
+      auto blocks_of = [&](int ti, int32_t *blk) { tile_blocks(p, b, static_cast<int64_t>(ti) * TILE, pc.vis, blk); };
+      auto rows_of = [&](int ti, const int32_t *blk, int32_t *r4) {
+        rows_of_blocks(p, b, static_cast<int64_t>(ti) * TILE, pc.vis, blk, r4);
+      };
+      int32_t cur[4], prev[4], nxt[4] = {0, 0, 0, 0}, raw0[4], raw[4] = {0, 0, 0, 0};
+      blocks_of(pc.t_begin, raw0);
+      if (pc.t_begin + 1 < pc.t_end) blocks_of(pc.t_begin + 1, raw);
+      rows_of(pc.t_begin, raw0, cur);
       if (w == Q_OWNER) {
         bool good = true;
         if (lane == 0) {
@@ -526,7 +536,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         }
       }
       for (int ti = pc.t_begin; ti < pc.t_end && ok; ++ti) {
-        if (ti + 1 < pc.t_end) rows_of(ti + 1, nxt);
+        if (ti + 1 < pc.t_end) {
+          rows_of(ti + 1, raw, nxt);
+          if (ti + 2 < pc.t_end) blocks_of(ti + 2, raw);
+        }
         const int32_t own[2] = {rank ? cur[2] : cur[0], rank ? cur[3] : cur[1]};
         if (!load_k(own)) { ok = false; break; }
         if (ti > pc.t_begin && !load_v(prev)) { ok = false; break; }
@@ -545,7 +558,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         const int uses = nbig > sl ? (nbig - sl + NBIG - 1) / NBIG : 0;
         if (uses > 0) mbar_wait(bar(BAR_BIG_EMPTY + sl), (uses - 1) & 1, abort_flag);
       }
-      if (ok && w == SMALL_OWNER && nsmall > 0) mbar_wait(bar(BAR_SMALL_EMPTY), (nsmall - 1) & 1, abort_flag);
+      if (ok && w == SMALL_OWNER && nsmall > 0)
+        mbar_wait(bar(BAR_S_FULL + ((nsmall - 1) & 1)), ((nsmall - 1) >> 1) & 1, abort_flag);
       if (ok && w == Q_OWNER && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
     }
   } else if (warp == WARP_MMA) {
@@ -565,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
           slot = 0;
           use = nsmall++;
         }
-        empty_bar = big ? BAR_BIG_EMPTY + slot : BAR_SMALL_EMPTY;
+        empty_bar = BAR_BIG_EMPTY + slot;  // (small items are released by S_FULL)
         if (!mbar_wait(bar(big ? BAR_BIG_FULL + slot : BAR_SMALL_FULL), use & 1, abort_flag)) return 0;
         tc_fence_after();
         return sbase + (big ? OFF_BIG + slot * BIG : OFF_SMALL);
@@ -593,9 +607,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
               ++gz;
               tc_fence_after();
             }
+            const uint64_t vd = sdesc_sw128(vb, ATOM, HALF);  // K step m: + 1024 bytes
 #pragma unroll
             for (int m = 0; m < 8; ++m)
-              tc_mma_ts<2>(tmem + 128 * j, p_col + 8 * (8 * vp + m), sdesc_sw128(vb + m * 1024, ATOM, HALF), IDESC_PV,
+              tc_mma_ts<2>(tmem + 128 * j, p_col + 8 * (8 * vp + m), sdesc_advance(vd, m * 1024), IDESC_PV,
                            (first && vp == 0 && m == 0) ? 0u : 1u);
             release();
           }
@@ -611,15 +626,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
             const bool big = q < K_ITEMS - 1;
             const uint32_t kbuf = take(big);
             if (kbuf == 0) { ok = false; break; }
+            // descriptors of the item's first K step; the others differ only in
+            // their start address (+32 bytes per K step, + a chunk per c)
+            const uint64_t qd = sdesc_sw128(sbase + OFF_Q + 2 * q * CHUNK_Q, 16, 1024);
+            const uint64_t kd = sdesc_sw128(kbuf, 16, 1024);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               if (!big && c == 1) break;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                tc_mma<2>(tmem + S_COL + 128 * b, sdesc_sw128(sbase + OFF_Q + (2 * q + c) * CHUNK_Q + kk * 32, 16, 1024),
-                          sdesc_sw128(kbuf + c * CHUNK_K + kk * 32, 16, 1024), IDESC_S, (q > 0 || c > 0 || kk > 0) ? 1u : 0u);
+                tc_mma<2>(tmem + S_COL + 128 * b, sdesc_advance(qd, c * CHUNK_Q + kk * 32),
+                          sdesc_advance(kd, c * CHUNK_K + kk * 32), IDESC_S, (q > 0 || c > 0 || kk > 0) ? 1u : 0u);
             }
-            release();
+            if (big) release();  // the small item is released by the S_FULL commit below
           }
           if (!ok) break;
           tc_commit_pair(bar(BAR_S_FULL + b), 0x3);
@@ -631,7 +650,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
         ++npc;
       }
     }
-  } else if (warp >= WARP_SOFTMAX) {
+  } else if (warp >= WARP_SOFTMAX && warp < WARP_SOFTMAX + 4) {
     // ------------------------------------------------- softmax + epilogue
     // A failed (timed-out) wait does not break these loops: every softmax
     // warp keeps the same sequence of named-barrier syncs and runs to the

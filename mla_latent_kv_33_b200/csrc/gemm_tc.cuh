@@ -262,11 +262,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
 //   q_lat,h = W_UK_h^T q_C,h (512 x T) -> q[t][h][j]
 // (MLA walk-through, section 1 step 3 and section 3 order B; DeepSeek-V2
 // explainer, eqs. 12-13.) Every CTA streams its head's 192 + 128 weight rows
-// once; q_C never leaves the SM. The q_R product runs as an M = 128 MMA whose
-// upper 64 rows read stale shared memory and are discarded.
+// once; q_C never leaves the SM. A stage holds the W_UQ box (128 rows), the
+// W_QR box (64 rows) and the c_Q box back to back; the q_R product runs as an
+// M = 128 MMA whose upper 64 rows read the c_Q box (or, for a small c_Q box,
+// whatever follows it in shared memory) into accumulator rows that are
+// discarded. Packing the 64-row box keeps 24 KB of weights in every 32 KB
+// stage (at T = 64), so six stages fit. While product 1 streams, the epilogue
+// warps fill a table of the RoPE cosines and sines of every (token, pair), so
+// that rotating q_R after it costs a few multiplies per element.
 namespace ab {
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB: a 128-row A tile (or two 64 x 64 W_UK^T boxes)
-constexpr int QR_BYTES = 64 * BK * 2;  // 8 KB loaded into a 16 KB slot
+constexpr int QR_BYTES = 64 * BK * 2;  // 8 KB
+// 8 warps: TMA producers 0, 6 and 7 (stage s is issued by producer s % 3), the
+// MMA warp 1, and the epilogue warps 2-5 (warp w reaches tensor-memory lanes
+// 32 (w % 4) .. + 31). A TMA instruction holds its issuing thread for a few
+// hundred ns, so one producer alone would cap the stage rate.
+constexpr int NUM_THREADS = 256, PRODUCERS = 3;
 struct Params {
   int T, n_tile, n_h, d_c, d_r, k_blocks;  // k_blocks = d_cq / 64
   int stages, stage_bytes, col_stride;      // col_stride: TMEM columns per accumulator
@@ -275,19 +286,22 @@ struct Params {
   double rope_base;
   int prefetch;  // launched with launch overlap: weight boxes of the first stages go out before griddep_wait
 };
+constexpr int RPAIRS = 32;  // RoPE pairs (d_R = 64)
 __host__ __device__ inline int b2_bytes(int n_tile) { return ((n_tile + 63) / 64) * 128 * 128; }
-inline int stage_bytes(int n_tile) { return 2 * A_BYTES + n_tile * BK * 2; }
+__host__ __device__ inline int tab_bytes(int n_tile) { return n_tile * RPAIRS * 8; }  // float2 (cos, sin) [t][pair]
+inline int stage_bytes(int n_tile) { return A_BYTES + QR_BYTES + n_tile * BK * 2; }
 inline int stages(int n_tile) {
-  const int budget = 200 * 1024 - b2_bytes(n_tile);
+  const int budget = 224 * 1024 - b2_bytes(n_tile) - tab_bytes(n_tile);
   const int s = budget / stage_bytes(n_tile);
   return s > 8 ? 8 : s;
 }
 inline size_t smem(int n_tile, int st) {
-  return static_cast<size_t>(st) * stage_bytes(n_tile) + b2_bytes(n_tile) + 8 * (2 * st + 3) + 16 + 1024;
+  return static_cast<size_t>(st) * stage_bytes(n_tile) + b2_bytes(n_tile) + tab_bytes(n_tile) + 8 * (2 * st + 3) + 16 +
+         1024;
 }
 }  // namespace ab
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(ab::NUM_THREADS, 1)
     k_absorb_head(const __grid_constant__ CUtensorMap tm_uq, const __grid_constant__ CUtensorMap tm_qr,
                   const __grid_constant__ CUtensorMap tm_cq, const __grid_constant__ CUtensorMap tm_uk,
                   const ab::Params p) {
@@ -297,12 +311,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x;
   const uint32_t b2 = sbase + p.stages * p.stage_bytes;  // q_C,h as the MN-major B of the second product
-  const uint32_t bars = b2 + ab::b2_bytes(p.n_tile);
+  float2 *rope_tab = reinterpret_cast<float2 *>(smem + p.stages * p.stage_bytes + ab::b2_bytes(p.n_tile));
+  const uint32_t bars = b2 + ab::b2_bytes(p.n_tile) + ab::tab_bytes(p.n_tile);
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   const uint32_t p1_done = bars + 8u * (2 * p.stages), b2_full = p1_done + 8, p2_done = p1_done + 16;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.stages * p.stage_bytes + ab::b2_bytes(p.n_tile) +
-                                                     8 * (2 * p.stages + 3));
+                                                     ab::tab_bytes(p.n_tile) + 8 * (2 * p.stages + 3));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const int n_p2 = 4 * 2;  // second product: 4 M tiles (512 latent rows) x 2 K blocks (d_h = 128)
 
@@ -324,13 +339,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer
-    // Under launch overlap the first stages are armed together and their
-    // weight boxes issued by lanes l (W_UQ or W_UK box 0) and 8 + l (W_QR or
-    // W_UK box 1) before the wait for the previous kernel on the stream;
-    // their c_Q boxes (lane l) only after it. Every other stage, in order:
-    // lane 0 waits and arms, lanes 0-2 issue.
+  if (warp == 0 || warp >= 6) {
+    // ------------------------------------------------------- TMA producers
+    // Under launch overlap the first stages are armed together by producer 0
+    // and their weight boxes issued by lanes l (W_UQ or W_UK box 0) and 8 + l
+    // (W_QR or W_UK box 1) before the wait for the previous kernel on the
+    // stream; their c_Q boxes (lane l) only after it. Every later use of stage
+    // s goes out from producer s % 3, in order (so each stage's empty-barrier
+    // waits are made by one warp): lane 0 waits and arms, lanes 0-2 issue.
+    const int pid = warp == 0 ? 0 : warp - 5;
     const int total = p.k_blocks + n_p2;
     const int pre = p.prefetch ? min(total, p.stages) : 0;  // stages <= 8
     auto stage_tx = [&](int g) { return g < p.k_blocks ? ab::A_BYTES + ab::QR_BYTES + p.n_tile * BK * 2 : ab::A_BYTES; };
@@ -348,19 +365,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     auto issue_cq = [&](int g) {
       const int s = g % p.stages;
-      tma_load_2d(sbase + s * p.stage_bytes + 2 * ab::A_BYTES, &tm_cq, g * BK, 0, full(s));
+      tma_load_2d(sbase + s * p.stage_bytes + ab::A_BYTES + ab::QR_BYTES, &tm_cq, g * BK, 0, full(s));
     };
-    if (lane == 0)
-      for (int g = 0; g < pre; ++g) mbar_arrive_expect_tx(full(g), stage_tx(g));
-    __syncwarp();
-    if (lane < pre) issue_w(lane, 0);
-    else if (lane >= 8 && lane - 8 < pre) issue_w(lane - 8, 1);
+    if (pid == 0) {
+      if (lane == 0)
+        for (int g = 0; g < pre; ++g) mbar_arrive_expect_tx(full(g), stage_tx(g));
+      __syncwarp();
+      if (lane < pre) issue_w(lane, 0);
+      else if (lane >= 8 && lane - 8 < pre) issue_w(lane - 8, 1);
+    }
     griddep_wait();
-    if (lane < pre && lane < p.k_blocks) issue_cq(lane);
+    if (pid == 0 && lane < pre && lane < p.k_blocks) issue_cq(lane);
     __syncwarp();
     int g = pre;
     for (; g < total; ++g) {
       const int s = g % p.stages;
+      if (s % ab::PRODUCERS != pid) continue;
       const bool first = g < p.k_blocks;
       bool good = true;
       if (lane == 0) {
@@ -372,9 +392,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else if (lane == 2 && first) issue_cq(g);
       __syncwarp();
     }
-    if (lane == 0)  // drain: the MMA commits to the empty barriers have landed
+    if (lane == 0)  // drain: the MMA commits to this producer's empty barriers have landed
       for (int q = g - p.stages; q < g; ++q)
-        if (q >= 0) mbar_wait(empty(q % p.stages), (q / p.stages) & 1, abort_flag);
+        if (q >= 0 && (q % p.stages) % ab::PRODUCERS == pid) mbar_wait(empty(q % p.stages), (q / p.stages) & 1, abort_flag);
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     const uint32_t id1 = idesc_bf16(BM, p.n_tile, false, false);
@@ -389,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t st = sbase + s * p.stage_bytes;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t bd = sdesc_sw128(st + 2 * ab::A_BYTES + kk * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(st + ab::A_BYTES + ab::QR_BYTES + kk * 32, 16, 1024);
         tc_mma<1>(d1, sdesc_sw128(st + kk * 32, 16, 1024), bd, id1, (g > 0 || kk > 0) ? 1u : 0u);
         tc_mma<1>(d2, sdesc_sw128(st + ab::A_BYTES + kk * 32, 16, 1024), bd, id1, (g > 0 || kk > 0) ? 1u : 0u);
       }
@@ -412,13 +432,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     tc_commit(p2_done);
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 6) {
     // ----------------------------------------------------------- epilogue
     const int sp = warp & 3;
     const int row = 32 * sp + lane;  // accumulator row of this thread
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
     const int64_t q_row = static_cast<int64_t>(p.n_h) * (p.d_c + p.d_r);  // q elements per token
     griddep_wait();  // positions are read and q written only once the previous kernel has finished
+    // RoPE table while product 1 streams: (cos, sin) of token t, pair i
+    for (int e = threadIdx.x - 64; e < p.n_tile * ab::RPAIRS; e += 128) {
+      const int t = e / ab::RPAIRS, i = e % ab::RPAIRS;
+      float c = 1.f, s = 0.f;
+      if (t < p.T) rope_cos_sin(p.positions[t], rope_theta(i, p.d_r, p.rope_base), c, s);
+      rope_tab[e] = make_float2(c, s);
+    }
+    named_bar_sync(1, 128);  // the four epilogue warps
     mbar_wait_warp(p1_done, 0, abort_flag);
     tc_fence_after();
     // q_C,h row `row` -> B2 (MN-major, 128-byte swizzle): k = row, n = token
@@ -442,7 +470,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // q_R,h rows 0..63 (warps of sub-partitions 0, 1): lanes (2k, 2k+1) hold a RoPE pair
     if (sp < 2) {
       const bool odd = (row & 1) != 0;
-      const double theta = rope_theta(row >> 1, p.d_r, p.rope_base);
       for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(lane_addr + p.col_stride + c0, v);
@@ -454,7 +481,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
           if (t < p.T) {
             float x0 = odd ? other : mine, x1 = odd ? mine : other;
-            rope_rotate(x0, x1, p.positions[t], theta);
+            const float2 cs = rope_tab[t * ab::RPAIRS + (row >> 1)];
+            rope_apply(x0, x1, cs.x, cs.y);
             p.q[t * q_row + static_cast<int64_t>(head) * (p.d_c + p.d_r) + p.d_c + row] = __float2bfloat16_rn(odd ? x1 : x0);
           }
         }

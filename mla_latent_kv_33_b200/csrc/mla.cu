@@ -608,7 +608,7 @@ mla_status tc_absorb_from_cq(const mla_dims *d, const __nv_bfloat16 *cq, const v
     if ((s = raise_smem_limit(reinterpret_cast<const void *>(G::k_absorb_head), SMEM_ABSORB, 232448,
                               "absorb: set shared memory size")) != MLA_OK)
       return s;
-    return launched(launch_tc(G::k_absorb_head, dim3(d->n_h), dim3(G::NUM_THREADS), smem, st, tq, tr, tc, tk, ap),
+    return launched(launch_tc(G::k_absorb_head, dim3(d->n_h), dim3(G::ab::NUM_THREADS), smem, st, tq, tr, tc, tk, ap),
                     "fused per-head absorb (tensor cores)");
   }
   // [q_C ; q_R] = [W_UQ ; W_QR] c_Q: q_C to the workspace, q_R rotated into q

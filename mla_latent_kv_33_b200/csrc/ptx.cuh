@@ -226,6 +226,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The descriptor of the operand `bytes` further on in shared memory: only the
+// 14-bit start-address field (address / 16, bits 0-13) changes. Shared-memory
+// addresses stay below 2^18 bytes, so the field never carries into the next.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // M, N are the whole instruction's extents (both CTAs for cta_group::2).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
