@@ -73,7 +73,9 @@ constexpr int TILE = 256, OWN = 128, BLK = 64;  // tokens per pair tile / per CT
 constexpr int NUM_PRODUCERS = 4, WARP_MMA = 3, WARP_SOFTMAX = 4, WARP_PROD3 = 8;
 constexpr int NUM_THREADS = 32 * 9;
 constexpr int NBIG = 4;              // 32 KB ring slots; big slot s belongs to producer s
-constexpr int SMALL_OWNER = 1, Q_OWNER = 2;
+// the small slot's producer; Q's three 24 KB boxes come from producers 0-2
+// (each waits Q's empty barrier for every piece, so each wait is exact)
+constexpr int SMALL_OWNER = 1, Q_LOADERS = 3;
 constexpr int CHUNK_Q = HPC * 128;   // 64 heads x 64 columns
 constexpr int ATOM = BLK * 128;      // 64 rows x 64 columns (one 128-byte-swizzle atom column)
 constexpr int CHUNK_K = 2 * ATOM;    // one column chunk of the CTA's 128 tokens
@@ -128,18 +130,32 @@ struct Params {
   float *part_o;    // [slots][128][512]
   float *part_lse;  // [slots][128]
   // [0] = W (visible tiles), [1] = Qt (tiles per cluster, automatic plan), [2] = splits,
-  // [3 ..] tile offsets of the rows [BJ + 1], then (splits > 0) piece offsets [BJ + 1]
+  // [3] = cluster groups G, [4] = clusters per group, [5 ..] tile offsets of the units
+  // [BJ + 1], then (splits > 0) piece offsets [BJ + 1]
   int32_t *plan;
   int32_t splits;   // 0: automatic plan; S > 0: every row in min(S, tiles) pieces
 };
 
 // Offsets of the plan arrays in Params::plan.
-__host__ __device__ constexpr int plan_tiles(int) { return 3; }
-__host__ __device__ constexpr int plan_pieces(int BJ) { return 4 + BJ; }
+__host__ __device__ constexpr int plan_tiles(int) { return 5; }
+__host__ __device__ constexpr int plan_pieces(int BJ) { return 6 + BJ; }
 
-// Tiles visible to unit bj (token row); -1 if its sequence length is invalid.
-__device__ __forceinline__ int unit_tiles(const Params &p, int bj, int *vis_out) {
-  const int b = bj / p.n_q, j = bj % p.n_q;
+// The tile line's units are the token rows in query-position-major order:
+// unit u = j B + b is row b n_q + j (new token j of sequence b). The kernel
+// is compiled twice: kGrouped = false serves n_q = 1, where unit and row
+// coincide, with none of the index arithmetic or cluster groups below.
+template <bool kGrouped>
+__device__ __forceinline__ int row_of_unit(const Params &p, int u) {
+  return !kGrouped ? u : (u % p.B) * p.n_q + u / p.B;
+}
+__device__ __forceinline__ int unit_of_row(const Params &p, int bj) {
+  return p.n_q == 1 ? bj : (bj % p.n_q) * p.B + bj / p.n_q;
+}
+
+// Tiles visible to unit u; -1 if its sequence length is invalid.
+template <bool kGrouped>
+__device__ __forceinline__ int unit_tiles(const Params &p, int u, int *vis_out) {
+  const int b = !kGrouped ? u : u % p.B, j = !kGrouped ? 0 : u / p.B;
   const int L = p.seq_lens[b];
   if (L < p.n_q || static_cast<int64_t>(L) > p.capacity) {
     *vis_out = 0;
@@ -201,23 +217,25 @@ __device__ __forceinline__ int split_piece_of(int r, int nt, int sp, int *end) {
 
 // Iterates the pieces of this cluster's tile range in order. Automatic plan:
 // pieces are cut by row ends and cluster boundaries, and the split slot of a
-// row's piece in cluster k is bj + k (a cluster holds at most one piece of a
-// row that continues into another cluster). Forced splits: pieces are also cut
-// at the row's piece boundaries, and the slot is the piece's global index.
+// unit's piece in cluster k is u + k (a cluster holds at most one piece of a
+// row that continues into another cluster); base is the first tile of the
+// cluster's group. Forced splits: pieces are also cut at the row's piece
+// boundaries, and the slot is the piece's global index.
+template <bool kGrouped>
 struct PieceIter {
-  int g, gend, bj, off, poff, Qt, k, S;
+  int g, gend, u, off, poff, Qt, k, S, base;
   __device__ bool next(const Params &p, Piece &pc) {
     while (g < gend) {
       int vis;
-      int nt = unit_tiles(p, bj, &vis);
+      int nt = unit_tiles<kGrouped>(p, u, &vis);
       if (nt < 0) nt = 0;
       if (nt == 0 || off + nt <= g) {
         off += nt;
         poff += S ? split_pieces(S, nt) : 0;
-        ++bj;
+        ++u;
         continue;
       }
-      pc.bj = bj;
+      pc.bj = row_of_unit<kGrouped>(p, u);
       pc.vis = vis;
       pc.nt = nt;
       pc.t_begin = g - off;
@@ -233,17 +251,17 @@ struct PieceIter {
         if (e == off + nt) {
           off += nt;
           poff += sp;
-          ++bj;
+          ++u;
         }
         return true;
       }
       const int e = min(gend, off + nt);
       pc.t_end = e - off;
-      pc.single = off / Qt == (off + nt - 1) / Qt;
-      pc.slot = bj + k;
+      pc.single = kGrouped ? (off - base) / Qt == (off + nt - 1 - base) / Qt : off / Qt == (off + nt - 1) / Qt;
+      pc.slot = u + k;
       g = e;
       off += nt;
-      ++bj;
+      ++u;
       return true;
     }
     return false;
@@ -320,6 +338,7 @@ __device__ __forceinline__ void arrive_leader(uint32_t bar_local, uint32_t rank)
     mbar_arrive_cluster(mapa_shared(bar_local, 0));
 }
 
+template <bool kGrouped>
 __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     k_decode(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v0,
@@ -339,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   int *ints = reinterpret_cast<int *>(misc + MISC_INTS);
   volatile int *abort_flag = ints + 0;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ints + 1);
-  int *plan_s = ints + 2;  // g0, g1, Qt, first row, its tile offset, its piece offset
+  int *plan_s = ints + 2;  // g0, g1, Qt, first unit, its tile offset, its piece offset, group base
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
@@ -378,9 +397,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   int *pieces = tiles + BJ;
   for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
     int vis;
-    int nt = unit_tiles(p, u, &vis);
+    int nt = unit_tiles<kGrouped>(p, u, &vis);
     if (nt < 0) {
-      if (blockIdx.x == 0 && (u % p.n_q) == 0) dev_error(MLA_DEVERR_DATA);
+      if (blockIdx.x == 0 && u < p.B) dev_error(MLA_DEVERR_DATA);  // once per sequence
       nt = 0;
     }
     tiles[u] = nt;
@@ -391,12 +410,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     __shared__ int warp_tot[NUM_THREADS / 32];
     const int W = block_exclusive_scan<NUM_THREADS>(tiles, BJ, warp_tot);
     const int P = S ? block_exclusive_scan<NUM_THREADS>(pieces, BJ, warp_tot) : 0;
+    // Automatic plan with n_q > 1 (and at least n_q clusters): one group of
+    // clusters per query position j cuts the line of the rows of position j
+    // into equal ranges, the same length Qt in every group, so that the n_q
+    // rows of a sequence stream the same cache tiles at about the same time
+    // and all but one of their reads hit L2.
+    const int G = kGrouped && S == 0 && nclusters >= p.n_q ? p.n_q : 1;
+    const int ncg = nclusters / G;
     if (threadIdx.x == 0) {
-      int g0, g1, Qt = 0;
+      int g0, g1, Qt = 0, base = 0;
       if (S == 0) {
-        Qt = max(1, (W + nclusters - 1) / nclusters);
-        g0 = min(W, cluster * Qt);
-        g1 = min(W, (cluster + 1) * Qt);
+        for (int q = 0; q < G; ++q) {
+          const int lo = G > 1 ? tiles[q * p.B] : 0, hi = q + 1 < G ? tiles[(q + 1) * p.B] : W;
+          Qt = max(Qt, (hi - lo + ncg - 1) / ncg);
+        }
+        Qt = max(1, Qt);
+        const int grp = cluster / ncg, kl = cluster % ncg;
+        if (grp < G) {
+          base = G > 1 ? tiles[grp * p.B] : 0;
+          const int end = grp + 1 < G ? tiles[(grp + 1) * p.B] : W;
+          g0 = min(end, base + kl * Qt);
+          g1 = min(end, base + (kl + 1) * Qt);
+        } else {
+          g0 = g1 = W;  // a cluster left over when n_q does not divide the clusters
+        }
       } else {
         const auto share = [&](int c) {
           return static_cast<int>((static_cast<int64_t>(c) * W + nclusters - 1) / nclusters);
@@ -411,6 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       plan_s[3] = u0;
       plan_s[4] = u0 < BJ ? tiles[u0] : W;
       plan_s[5] = S && u0 < BJ ? pieces[u0] : 0;
+      plan_s[6] = base;
     }
     if (blockIdx.x == 0) {  // the layout k_combine reads
       for (int u = threadIdx.x; u < BJ; u += NUM_THREADS) {
@@ -419,8 +457,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       }
       if (threadIdx.x == 0) {
         p.plan[0] = W;
-        p.plan[1] = S == 0 ? max(1, (W + nclusters - 1) / nclusters) : 0;
+        p.plan[1] = S == 0 ? max(1, plan_s[2]) : 0;
         p.plan[2] = S;
+        p.plan[3] = G;
+        p.plan[4] = ncg;
         p.plan[plan_tiles(BJ) + BJ] = W;
         if (S) p.plan[plan_pieces(BJ) + BJ] = P;
       }
@@ -431,15 +471,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
   cluster_sync_all();  // peer barriers initialised, TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  PieceIter it0;
+  PieceIter<kGrouped> it0;
   it0.g = plan_s[0];
   it0.gend = plan_s[1];
   it0.Qt = max(1, plan_s[2]);
-  it0.bj = plan_s[3];
+  it0.u = plan_s[3];
   it0.off = plan_s[4];
   it0.poff = plan_s[5];
   it0.k = cluster;
   it0.S = S;
+  it0.base = plan_s[6];
 
   if (warp < WARP_MMA || warp == WARP_PROD3) {
     // --------------------------------------------------------- ring producers
@@ -450,7 +491,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     // arms its full barrier, then lane l issues box l of the item.
     const int w = warp < WARP_MMA ? warp : 3;  // producer index
     const uint32_t q_full = rank == 0 ? bar(BAR_Q_FULL) : mapa_shared(bar(BAR_Q_FULL), 0);
-    PieceIter it = it0;
+    PieceIter<kGrouped> it = it0;
     Piece pc;
     int nbig = 0, nsmall = 0, npc = 0;
     bool ok = true;
@@ -521,13 +562,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       blocks_of(pc.t_begin, raw0);
       if (pc.t_begin + 1 < pc.t_end) blocks_of(pc.t_begin + 1, raw);
       rows_of(pc.t_begin, raw0, cur);
-      if (w == Q_OWNER) {
+      if (w < Q_LOADERS) {  // producer w loads Q's column chunks 3 w .. 3 w + 2
         bool good = true;
         if (lane == 0) {
           if (npc > 0) good = mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
           if (good) {
-            if (rank == 0) mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * Q_BYTES);
-            tma_load_3d_pair(sbase + OFF_Q, &tm_q, 0, pc.bj * HEADS + HPC * rank, 0, q_full);
+            if (rank == 0 && w == 0) mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * Q_BYTES);
+            tma_load_3d_pair(sbase + OFF_Q + 3 * w * CHUNK_Q, &tm_q, 0, pc.bj * HEADS + HPC * rank, 3 * w, q_full);
           }
         }
         if (!__shfl_sync(0xffffffffu, good, 0)) {
@@ -560,12 +601,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
       }
       if (ok && w == SMALL_OWNER && nsmall > 0)
         mbar_wait(bar(BAR_S_FULL + ((nsmall - 1) & 1)), ((nsmall - 1) >> 1) & 1, abort_flag);
-      if (ok && w == Q_OWNER && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
+      if (ok && w < Q_LOADERS && npc > 0) mbar_wait(bar(BAR_Q_EMPTY), (npc - 1) & 1, abort_flag);
     }
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0) {
-      PieceIter it = it0;
+      PieceIter<kGrouped> it = it0;
       Piece pc{};
       int gi = 0, nbig = 0, nsmall = 0, gz = 0, npc = 0, empty_bar = 0;
       bool ok = true;
@@ -660,7 +701,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     const int row = L & 63, half = L >> 6;  // head within CTA; token half / latent half
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
     const float c2 = p.scale_log2;
-    PieceIter it = it0;
+    PieceIter<kGrouped> it = it0;
     Piece pc;
     int gi = 0, gz = 0, bbase = 0;  // bbase: big-slot uses before this piece
     while (it.next(p, pc)) {
@@ -867,20 +908,23 @@ constexpr int COMBINE_CHUNK = 2, COMBINE_BLOCKS_PER_ROW = HEADS / 4;
 __global__ void __launch_bounds__(128) k_combine(Params p) {
   if (threadIdx.x == 0) griddep_launch_dependents();
   griddep_wait();
-  const int bj = blockIdx.x / COMBINE_BLOCKS_PER_ROW;
+  const int bj = blockIdx.x / COMBINE_BLOCKS_PER_ROW;  // token row
   const int head = 4 * (blockIdx.x % COMBINE_BLOCKS_PER_ROW) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int BJ = p.B * p.n_q;
+  const int u = unit_of_row(p, bj);
   int first, np;
-  if (p.plan[2] == 0) {  // automatic plan: the row's pieces are its clusters k0 .. k1, slots bj + k
-    const int a = p.plan[plan_tiles(BJ) + bj], e = p.plan[plan_tiles(BJ) + bj + 1], Qt = p.plan[1];
+  if (p.plan[2] == 0) {  // automatic plan: the unit's pieces are its clusters k0 .. k1, slots u + k
+    const int G = p.plan[3], ncg = p.plan[4], grp = G > 1 ? u / p.B : 0;
+    const int base = G > 1 ? p.plan[plan_tiles(BJ) + grp * p.B] : 0, Qt = p.plan[1];
+    const int a = p.plan[plan_tiles(BJ) + u] - base, e = p.plan[plan_tiles(BJ) + u + 1] - base;
     if (e <= a) return;
-    const int k0 = a / Qt, k1 = (e - 1) / Qt;
-    first = bj + k0;
+    const int k0 = grp * ncg + a / Qt, k1 = grp * ncg + (e - 1) / Qt;
+    first = u + k0;
     np = k1 - k0 + 1;
-  } else {  // forced splits: the row's pieces are slots piece_off[bj] ..
-    first = p.plan[plan_pieces(BJ) + bj];
-    np = p.plan[plan_pieces(BJ) + bj + 1] - first;
+  } else {  // forced splits: the unit's pieces are slots piece_off[u] ..
+    first = p.plan[plan_pieces(BJ) + u];
+    np = p.plan[plan_pieces(BJ) + u + 1] - first;
   }
   if (np <= 1) return;
   const float *pl = p.part_lse + static_cast<int64_t>(first) * HEADS + head;
@@ -950,7 +994,7 @@ __global__ void __launch_bounds__(128) k_combine(Params p) {
 // row boundaries), then fp32 split partials. Slots: at most BJ + clusters for
 // the automatic plan; for S forced splits at most BJ * min(S, tiles of the
 // longest row), max_seq_len (0 = unknown) bounding the tiles.
-constexpr size_t decode_plan_bytes(size_t BJ) { return ((2 * BJ + 5) * sizeof(int32_t) + 255) & ~size_t(255); }
+constexpr size_t decode_plan_bytes(size_t BJ) { return ((2 * BJ + 7) * sizeof(int32_t) + 255) & ~size_t(255); }
 inline size_t decode_tc_slots(int B, int n_q, int sms, int splits, int64_t max_seq_len) {
   const size_t BJ = static_cast<size_t>(B) * n_q;
   size_t slots = BJ + static_cast<size_t>(sms / 2);

@@ -87,7 +87,7 @@ mla_status launched(cudaError_t e, const char *what) {
 
 // cudaFuncSetAttribute applies to the current device: a kernel's dynamic
 // shared memory limit is raised once per device (bit `device` of its mask).
-enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_ATTEND_A = 3, SMEM_KERNELS = 4 };
+enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_ATTEND_A = 3, SMEM_DECODE_NQ = 4, SMEM_KERNELS = 5 };
 std::atomic<uint64_t> g_smem_raised[SMEM_KERNELS];
 
 mla_status raise_smem_limit(const void *kernel, SmemKernel which, int bytes, const char *what) {
@@ -1051,7 +1051,7 @@ int decode_clusters(int sms) {
     if (c > 0) return std::min(c, sms / 2);
   }
   namespace D = mla::dec;
-  cudaFuncSetAttribute(D::k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES);
+  cudaFuncSetAttribute(D::k_decode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_BYTES);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
   cfg.blockDim = dim3(D::NUM_THREADS, 1, 1);
@@ -1064,7 +1064,7 @@ int decode_clusters(int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, D::k_decode, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, D::k_decode<false>, &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = sms / 2;
   }
@@ -1088,7 +1088,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
     return fail(MLA_ERR_WORKSPACE, "decode workspace too small");
 
   // Views of q and the cache (rows of 576 bf16 = 1152 bytes):
-  //   q:        (64 cols, row, 9 chunks of 128 B)        box (64, 64 heads, 9)
+  //   q:        (64 cols, row, 9 chunks of 128 B)        box (64, 64 heads, 3): a third of a CTA's Q
   //   score:    (576 cols, row)                          box (64, 64 tokens): one column chunk of a block
   //   value:    (64 cols, row, 2 chunks, 2 halves) at column 128 * rank, half stride 256 cols
   //             box (64, 64 tokens, 2, 1) = 128 of this CTA's latent columns of a block
@@ -1097,7 +1097,7 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   const uint64_t row_b = D::D * 2;
   {
     const uint64_t dims[3] = {64, static_cast<uint64_t>(BJ) * D::HEADS, 9}, str[2] = {row_b, 128};
-    const uint32_t box[3] = {64, D::HPC, 9};
+    const uint32_t box[3] = {64, D::HPC, 3};
     if ((s = make_tmap_nd(&tm_q, q, 3, dims, str, box, "q")) != MLA_OK) return s;
   }
   {
@@ -1135,11 +1135,13 @@ mla_status decode_tc(const mla_dims *d, const void *q, const mla_cache *c, const
   p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + plan_bytes);
   p.part_lse = p.part_o + slots * D::HEADS * D::DC;
 
-  if ((s = raise_smem_limit(reinterpret_cast<const void *>(D::k_decode), SMEM_DECODE, D::SMEM_BYTES,
-                            "decode: set shared memory size")) != MLA_OK)
+  // n_q > 1: the variant whose cluster groups follow the query positions
+  const auto kernel = n_q > 1 ? D::k_decode<true> : D::k_decode<false>;
+  if ((s = raise_smem_limit(reinterpret_cast<const void *>(kernel), n_q > 1 ? SMEM_DECODE_NQ : SMEM_DECODE,
+                            D::SMEM_BYTES, "decode: set shared memory size")) != MLA_OK)
     return s;
-  if ((s = launched(launch_tc(D::k_decode, dim3(2 * nclusters), dim3(D::NUM_THREADS), D::SMEM_BYTES, st, tm_q,
-                              tm_k, tm_v[0], tm_v[1], p),
+  if ((s = launched(launch_tc(kernel, dim3(2 * nclusters), dim3(D::NUM_THREADS), D::SMEM_BYTES, st, tm_q, tm_k, tm_v[0],
+                              tm_v[1], p),
                     "decode (tensor cores)")) != MLA_OK)
     return s;
   return launched(launch_tc(D::k_combine, dim3(BJ * D::COMBINE_BLOCKS_PER_ROW), dim3(128), 0, st, p),
