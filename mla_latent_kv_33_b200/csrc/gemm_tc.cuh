@@ -18,7 +18,11 @@
 namespace mla {
 namespace gemm {
 
-constexpr int BM = 128, BK = 64, NUM_THREADS = 192;
+// k_gemm: TMA producer warps 0, 6 and 7 (stage s is issued by producer s % 3),
+// the MMA warp 1, the epilogue warps 2-5. The TMA operations one warp issues
+// complete one after another (~50 GB/s per warp), so a CTA that must stream
+// its operands faster needs several issuing warps.
+constexpr int BM = 128, BK = 64, NUM_THREADS = 256, PRODUCERS = 3;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 
 // Epilogue of one GEMM launch.
@@ -110,15 +114,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   const CUtensorMap *am = third ? &tm_a3 : (second ? &tm_a2 : &tm_a);
   const int am0 = third ? m0 - p.m_split2 : (second ? m0 - p.m_split : m0);
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    // A TMA instruction holds its issuing thread for ~0.3 us, but lanes issue
-    // in parallel, so every box goes out from its own lane. Under launch
-    // overlap the first stages are armed together and their weight boxes
-    // issued before the wait for the previous kernel on the stream (weights
-    // do not depend on it), their token boxes after it. Otherwise the stages
-    // go out in order, each stage's boxes together, so that the first stage
-    // is not queued behind the weights of all the others.
+  if (warp == 0 || warp >= 6) {
+    // --------------------------------------------------------- TMA producers
+    // Every use of stage s is issued by producer s % 3, in order (so each
+    // stage's empty-barrier waits are made by one warp). Under launch overlap
+    // the first stages are armed together and their weight boxes issued before
+    // the wait for the previous kernel on the stream (weights do not depend on
+    // it), their token boxes after it. Otherwise the stages go out in order,
+    // each stage's boxes together, so that the first stage is not queued
+    // behind the weights of all the others.
+    const int pid = warp == 0 ? 0 : warp - 5;
     const uint32_t stage0 = sbase;
     auto issue_a = [&](int i, int box) {  // box 1: second 64-wide m box of an MN-major A
       const uint32_t a_dst = stage0 + (i % p.stages) * stage_bytes;
@@ -139,17 +144,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       }
     };
     const int nkp = p.idle_producer ? 0 : nkb;  // self-test: nothing is issued, no copy is in flight
-    const int pre = p.prefetch ? min(nkp, p.stages) : 0;  // stages <= 12: lanes l and 16 + l serve stage l
+    // stages <= 12: lanes l and 16 + l serve this producer's l-th early stage
+    const int pre = p.prefetch ? min(nkp, p.stages) : 0;
+    const int ip = pid + PRODUCERS * (lane & 15);
     if (lane == 0)
-      for (int i = 0; i < pre; ++i) mbar_arrive_expect_tx(full(i), stage_bytes);
+      for (int i = pid; i < pre; i += PRODUCERS) mbar_arrive_expect_tx(full(i), stage_bytes);
     __syncwarp();
-    if (lane < pre) issue_a(lane, 0);
-    else if (lane >= 16 && lane - 16 < pre && p.a_mn_major) issue_a(lane - 16, 1);
+    if (ip < pre) {
+      if (lane < 16) issue_a(ip, 0);
+      else if (p.a_mn_major) issue_a(ip, 1);
+    }
     griddep_wait();
-    if (lane < pre) issue_b(lane);
+    if (lane < 16 && ip < pre) issue_b(ip);
     __syncwarp();
     for (int i = pre; i < nkp; ++i) {
       const int s = i % p.stages;
+      if (s % PRODUCERS != pid) continue;
       bool good = true;
       if (lane == 0) {
         if (i >= p.stages) good = mbar_wait(empty(s), ((i / p.stages) - 1) & 1, abort_flag, wait_ns);
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       tc_commit(empty(s));
     }
     tc_commit(done);
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------- epilogue
     const int sp = warp & 3;
     const int row = 32 * sp + lane;  // m within tile
@@ -277,7 +287,7 @@ constexpr int QR_BYTES = 64 * BK * 2;  // 8 KB
 // MMA warp 1, and the epilogue warps 2-5 (warp w reaches tensor-memory lanes
 // 32 (w % 4) .. + 31). A TMA instruction holds its issuing thread for a few
 // hundred ns, so one producer alone would cap the stage rate.
-constexpr int NUM_THREADS = 256, PRODUCERS = 3;
+constexpr int NUM_THREADS = 256;
 struct Params {
   int T, n_tile, n_h, d_c, d_r, k_blocks;  // k_blocks = d_cq / 64
   int stages, stage_bytes, col_stride;      // col_stride: TMEM columns per accumulator
@@ -380,7 +390,7 @@ __global__ void __launch_bounds__(ab::NUM_THREADS, 1)
     int g = pre;
     for (; g < total; ++g) {
       const int s = g % p.stages;
-      if (s % ab::PRODUCERS != pid) continue;
+      if (s % PRODUCERS != pid) continue;
       const bool first = g < p.k_blocks;
       bool good = true;
       if (lane == 0) {
@@ -394,7 +404,7 @@ __global__ void __launch_bounds__(ab::NUM_THREADS, 1)
     }
     if (lane == 0)  // drain: the MMA commits to this producer's empty barriers have landed
       for (int q = g - p.stages; q < g; ++q)
-        if (q >= 0 && (q % p.stages) % ab::PRODUCERS == pid) mbar_wait(empty(q % p.stages), (q / p.stages) & 1, abort_flag);
+        if (q >= 0 && (q % p.stages) % PRODUCERS == pid) mbar_wait(empty(q % p.stages), (q / p.stages) & 1, abort_flag);
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     const uint32_t id1 = idesc_bf16(BM, p.n_tile, false, false);

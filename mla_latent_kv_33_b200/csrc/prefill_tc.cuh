@@ -113,37 +113,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int kmax = bad || j0 >= p.n_q ? 0 : L - p.n_q + jl + 1;
   const int n = (kmax + KTILE - 1) / KTILE;  // key tiles (0: nothing to do)
 
-  if (warp == WARP_PROD) {
-    // ------------------------------------------------------------ producer
+  if (warp == WARP_PROD || warp == 2 || warp == 3) {
+    // ----------------------------------------------------------- producers
+    // TMA operations issued by one warp complete one after another, so the
+    // loads of a key tile come from three warps: warp 0 loads Q and the K_C
+    // chunks, warp 3 the k_R chunk (both fill the K slot: each waits for it
+    // to be free, warp 0 arms it), warp 2 the V tile.
+    const int role = warp == WARP_PROD ? 0 : (warp == 2 ? 1 : 2);  // 0: Q + K_C, 1: V, 2: k_R
     if (lane == 0 && n > 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(bar(BAR_Q), Q_BYTES);
-      for (int c = 0; c < 3; ++c)  // q rows b n_q + j0 .. (+128), head h; rows past T read zeros
-        tma_load_3d(sbase + OFF_Q + c * CHUNK, &tm_q, 64 * c, h, b * p.n_q + j0, bar(BAR_Q));
+      if (role == 0) {
+        mbar_arrive_expect_tx(bar(BAR_Q), Q_BYTES);
+        for (int c = 0; c < 3; ++c)  // q rows b n_q + j0 .. (+128), head h; rows past T read zeros
+          tma_load_3d(sbase + OFF_Q + c * CHUNK, &tm_q, 64 * c, h, b * p.n_q + j0, bar(BAR_Q));
+      }
       for (int i = 0; i < n && ok; ++i) {
         const int s = i & 1, use = i >> 1;
         int32_t r[2];
         for (int kb = 0; kb < 2; ++kb) r[kb] = block_row(p, b, static_cast<int64_t>(i) * KTILE + BLK * kb, L);
-        if (use > 0 && !mbar_wait(bar(BAR_KE + s), (use - 1) & 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(BAR_KF + s), K_BYTES);
-        const uint32_t kd = sbase + OFF_K + s * K_BYTES;
-        for (int kb = 0; kb < 2; ++kb) {
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(kd + c * CHUNK + kb * (CHUNK / 2), &tm_kc, 64 * c, r[kb], h, bar(BAR_KF + s));
-          tma_load_2d(kd + 2 * CHUNK + kb * (CHUNK / 2), &tm_kr, 512, r[kb], bar(BAR_KF + s));
+        if (role != 1) {
+          if (use > 0 && !mbar_wait(bar(BAR_KE + s), (use - 1) & 1, abort_flag)) { ok = false; break; }
+          const uint32_t kd = sbase + OFF_K + s * K_BYTES;
+          if (role == 0) {
+            mbar_arrive_expect_tx(bar(BAR_KF + s), K_BYTES);
+            for (int kb = 0; kb < 2; ++kb)
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d(kd + c * CHUNK + kb * (CHUNK / 2), &tm_kc, 64 * c, r[kb], h, bar(BAR_KF + s));
+          } else {
+            for (int kb = 0; kb < 2; ++kb)
+              tma_load_2d(kd + 2 * CHUNK + kb * (CHUNK / 2), &tm_kr, 512, r[kb], bar(BAR_KF + s));
+          }
+        } else {
+          if (use > 0 && !mbar_wait(bar(BAR_VE + s), (use - 1) & 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(BAR_VF + s), V_BYTES);
+          const uint32_t vd = sbase + OFF_V + s * V_BYTES;
+          for (int kb = 0; kb < 2; ++kb)
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(vd + c * CHUNK + kb * (CHUNK / 2), &tm_v, 64 * c, r[kb], h, bar(BAR_VF + s));
         }
-        if (use > 0 && !mbar_wait(bar(BAR_VE + s), (use - 1) & 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(BAR_VF + s), V_BYTES);
-        const uint32_t vd = sbase + OFF_V + s * V_BYTES;
-        for (int kb = 0; kb < 2; ++kb)
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(vd + c * CHUNK + kb * (CHUNK / 2), &tm_v, 64 * c, r[kb], h, bar(BAR_VF + s));
       }
-      // drain: the MMA's releases of the last use of each slot have arrived
-      for (int i = max(0, n - 2); ok && i < n; ++i) {
-        mbar_wait(bar(BAR_KE + (i & 1)), (i >> 1) & 1, abort_flag);
-        mbar_wait(bar(BAR_VE + (i & 1)), (i >> 1) & 1, abort_flag);
-      }
+      // drain: the MMA's releases of the last use of each slot this warp fills have arrived
+      for (int i = max(0, n - 2); ok && i < n; ++i)
+        mbar_wait(bar((role != 1 ? BAR_KE : BAR_VE) + (i & 1)), (i >> 1) & 1, abort_flag);
     }
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
