@@ -87,7 +87,9 @@ mla_status launched(cudaError_t e, const char *what) {
 
 // cudaFuncSetAttribute applies to the current device: a kernel's dynamic
 // shared memory limit is raised once per device (bit `device` of its mask).
-enum SmemKernel { SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_ATTEND_A = 3, SMEM_DECODE_NQ = 4, SMEM_KERNELS = 5 };
+enum SmemKernel {
+  SMEM_GEMM = 0, SMEM_ABSORB = 1, SMEM_DECODE = 2, SMEM_ATTEND_A = 3, SMEM_DECODE_NQ = 4, SMEM_GEMM_RES = 5, SMEM_KERNELS = 6
+};
 std::atomic<uint64_t> g_smem_raised[SMEM_KERNELS];
 
 mla_status raise_smem_limit(const void *kernel, SmemKernel which, int bytes, const char *what) {
@@ -896,24 +898,30 @@ mla_status tc_attend_a(const mla_dims *d, const void *qa, const void *W_UK, cons
   __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(w8);
   __nv_bfloat16 *vv = reinterpret_cast<__nv_bfloat16 *>(w8 + align256(static_cast<size_t>(d->n_h) * R * d->d_h * 2));
   mla_status s;
-  // decompression over every physical cache row: X_h[r][i] = sum_j W[h d_h + i][j] c_KV[r][j]
-  const GemmShape g = gemm_shape(d->d_h, static_cast<int>(R), d->d_c, d->n_h, false);
-  CUtensorMap tb;
-  if ((s = make_tmap_bf16(&tb, c->data, d->d_c, R, D * 2, 64, g.n_tile, "cache (c_KV)")) != MLA_OK) return s;
-  const void *Ws[2] = {W_UK, W_UV};
+  // decompression over every physical cache row, K_C and V in one launch:
+  // X_h[r][i] = sum_j W[h d_h + i][j] c_KV[r][j] for W = W_UK, W_UV
   __nv_bfloat16 *dsts[2] = {kc, vv};
-  for (int u = 0; u < 2; ++u) {
-    CUtensorMap ta;
-    if ((s = make_tmap_bf16(&ta, Ws[u], d->d_c, HD, d->d_c * 2ull, 64, 128, u == 0 ? "W_UK" : "W_UV")) != MLA_OK)
+  {
+    CUtensorMap ta0, ta1, tx;
+    if ((s = make_tmap_bf16(&tx, c->data, d->d_c, R, D * 2, 64, G::rs::NT, "cache (c_KV)")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&ta0, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UK")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&ta1, W_UV, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UV")) != MLA_OK) return s;
+    G::rs::Params rp{};
+    rp.batches = 2 * d->n_h;
+    rp.split = d->n_h;
+    rp.n_tiles = static_cast<int>((R + G::rs::NT - 1) / G::rs::NT);
+    rp.N = static_cast<int>(R);
+    rp.kblk = d->d_c / G::BK;
+    rp.out0 = kc;
+    rp.out1 = vv;
+    const int grid = std::max(1, std::min(sm_count(), rp.batches * rp.n_tiles));
+    if ((s = raise_smem_limit(reinterpret_cast<const void *>(G::k_gemm_resident), SMEM_GEMM_RES, G::rs::SMEM_BYTES,
+                              "decompression: set shared memory size")) != MLA_OK)
       return s;
-    G::Params p{};
-    p.epi = G::EPI_BF16;
-    p.dst = dsts[u];
-    p.e_bs = R * d->d_h;
-    p.e_ns = d->d_h;
-    GemmOperands op = operands(ta, tb);
-    op.a_batch_rows = d->d_h;
-    if ((s = launch_gemm(op, g, static_cast<int>(R), p, st)) != MLA_OK) return s;
+    if ((s = launched(launch_tc(G::k_gemm_resident, dim3(grid), dim3(G::rs::NUM_THREADS), G::rs::SMEM_BYTES, st, ta0,
+                                ta1, tx, rp),
+                      "order-A decompression (tensor cores)")) != MLA_OK)
+      return s;
   }
   // attention
   const int T = B * n_q;
