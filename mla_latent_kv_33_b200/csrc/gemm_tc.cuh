@@ -531,135 +531,156 @@ __global__ void __launch_bounds__(ab::NUM_THREADS, 1)
 // 128, n < N, k < K (a multiple of 64, 192 <= K <= 512), bf16 out, fp32
 // accumulation. This is the decompression of order A (MLA walk-through,
 // section 3 order A: K_C,h = W_UK,h c_KV and V_h = W_UV,h c_KV for every
-// cached row; X = the c_KV columns of the cache rows), a long run of
-// 128 x 256 tiles that share A within a batch. A persistent CTA per SM takes
-// a contiguous range of (batch, 256-row tile) pairs: the batch's A (128 x K,
-// up to 128 KB) stays in shared memory, X tiles stream through a three-slot
-// ring, and the two tensor-memory accumulators alternate so that the
-// epilogue of one tile overlaps the MMAs of the next.
+// cached row; X = the c_KV columns of the cache rows), a long run of tiles
+// that share A within a batch and X across batches.
+//
+// A pair of SMs (a 2-CTA cluster) takes batches 2c and 2c + 1 together: CTA r
+// keeps batch 2c + r's A (128 x K, up to 128 KB) in shared memory and loads
+// rows [128 r, 128 r + 128) of each 256-row X tile, and one
+// tcgen05.mma.cta_group::2 with M = 256, N = 256 multiplies both heads by the
+// whole tile, so every X byte read serves two heads. Each cluster takes a
+// contiguous range of (batch pair, 256-row tile) units; X half-tiles stream
+// through a six-slot ring, and two tensor-memory accumulators alternate so
+// that the epilogue of one tile overlaps the MMAs of the next. Eight epilogue
+// warps, two per tensor-memory sub-partition (one per half of the columns),
+// drain a tile in about half the time the MMAs of the next one take.
 namespace rs {
-constexpr int KBLK_MAX = 8, NT = 256, STAGES = 3, NUM_THREADS = 256;
-constexpr int A_BLK = BM * BK * 2;   // 16 KB: 128 rows x 64 k
-constexpr int B_STAGE = NT * BK * 2;  // 32 KB: 256 rows x 64 k
+// warps: producers 0, 6, 7; MMA 1; epilogue 2-5 and 8-11 (warp w reaches lanes 32 (w % 4) .. + 31)
+constexpr int KBLK_MAX = 8, NT = 256, NHALF = 128, STAGES = 6, NUM_THREADS = 384, EPI_WARPS = 8;
+constexpr int A_BLK = BM * BK * 2;       // 16 KB: 128 rows x 64 k
+constexpr int B_STAGE = NHALF * BK * 2;  // 16 KB: this CTA's 128 rows x 64 k
 constexpr int OFF_B = KBLK_MAX * A_BLK, OFF_BAR = OFF_B + STAGES * B_STAGE;
 constexpr int BAR_A_FULL = 0, BAR_A_EMPTY = 1, BAR_B_FULL = 2, BAR_B_EMPTY = BAR_B_FULL + STAGES,
-              BAR_ACC_FULL = BAR_B_EMPTY + STAGES, BAR_ACC_EMPTY = BAR_ACC_FULL + 2, NUM_BARS = BAR_ACC_EMPTY + 2;
+              BAR_ACC_FULL = BAR_B_EMPTY + STAGES, BAR_ACC_EMPTY = BAR_ACC_FULL + 2, BAR_EXIT = BAR_ACC_EMPTY + 2,
+              NUM_BARS = BAR_EXIT + 1;
 constexpr int SMEM_BYTES = OFF_BAR + 8 * NUM_BARS + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "resident-A GEMM shared memory budget");
-static_assert(STAGES == PRODUCERS, "one producer warp per ring slot");
+static_assert(STAGES % PRODUCERS == 0, "each producer owns whole ring slots");
 struct Params {
-  int batches, split;  // batches < split read A map 0, the rest A map 1
+  int batches, split;  // batches (even) < split read A map 0, the rest A map 1
   int n_tiles, N;      // 256-row tiles per batch, rows of X
   int kblk;            // K / 64
   __nv_bfloat16 *out0, *out1;  // [split][N][128] each
 };
 }  // namespace rs
 
-__global__ void __launch_bounds__(rs::NUM_THREADS, 1)
+__global__ void __launch_bounds__(rs::NUM_THREADS, 1) __cluster_dims__(2, 1, 1)
     k_gemm_resident(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                     const __grid_constant__ CUtensorMap tm_x, const rs::Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
+  const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bars = sbase + rs::OFF_BAR;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  auto lead = [&](int i) { return rank == 0 ? bar(i) : mapa_shared(bar(i), 0); };  // the leader CTA's barrier
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + rs::OFF_BAR + 8 * rs::NUM_BARS);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  const int total = p.batches * p.n_tiles;
-  const int t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * total / gridDim.x);
-  const int t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * total / gridDim.x);
-  auto batch_start = [&](int t) { return t == t0 || t % p.n_tiles == 0; };
+  const int units = (p.batches / 2) * p.n_tiles, cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int u0 = static_cast<int>(static_cast<int64_t>(cluster) * units / nclusters);
+  const int u1 = static_cast<int>(static_cast<int64_t>(cluster + 1) * units / nclusters);
+  auto pair_start = [&](int u) { return u == u0 || u % p.n_tiles == 0; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < rs::NUM_BARS; ++i) mbar_init(bar(i), i >= rs::BAR_ACC_EMPTY ? 4 : 1);
+    for (int i = 0; i < rs::NUM_BARS; ++i)
+      mbar_init(bar(i), i == rs::BAR_ACC_EMPTY || i == rs::BAR_ACC_EMPTY + 1 ? 2 * rs::EPI_WARPS : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc<1>(smem_u32(tmem_slot), 512);
+  if (warp == 1) tmem_alloc<2>(smem_u32(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // barriers initialised and tensor memory allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == 0 || warp >= 6) {
+  if (warp == 0 || warp == 6 || warp == 7) {
     // ---------------------------------------------------------- producers
-    // Producer q owns ring slot q; the A boxes of a batch are shared out
-    // (kb = q, q + 3, ..), each producer waiting for the previous A to be
-    // released, so every A phase needs every producer and each wait is exact.
+    // Producer q owns ring slots q and q + 3 of this CTA. The A boxes of a
+    // batch are shared out (kb = q, q + 3, ..), each producer waiting for the
+    // previous A to be released, so every A phase needs every producer and
+    // each wait is exact. Loads complete on the leader CTA's full barriers,
+    // which the leader's producer 0 (A) or slot owner (X) arms for both CTAs.
     const int pid = warp == 0 ? 0 : warp - 5;
     griddep_wait();  // the cache rows may come from the kernel ahead on the stream
     if (lane == 0) {
       int na = 0, g = 0;
       bool ok = true;
-      for (int t = t0; t < t1 && ok; ++t) {
-        const int b = t / p.n_tiles, nt = t % p.n_tiles;
-        if (batch_start(t)) {
+      for (int u = u0; u < u1 && ok; ++u) {
+        const int bp = u / p.n_tiles, nt = u % p.n_tiles, b = 2 * bp + static_cast<int>(rank);
+        if (pair_start(u)) {
           if (na > 0) ok = mbar_wait(bar(rs::BAR_A_EMPTY), (na - 1) & 1, abort_flag);
           if (!ok) break;
-          if (pid == 0) mbar_arrive_expect_tx(bar(rs::BAR_A_FULL), p.kblk * rs::A_BLK);
+          if (pid == 0 && rank == 0) mbar_arrive_expect_tx(bar(rs::BAR_A_FULL), 2 * p.kblk * rs::A_BLK);
           const CUtensorMap *am = b < p.split ? &tm_a0 : &tm_a1;
           const int h = b < p.split ? b : b - p.split;
           for (int kb = pid; kb < p.kblk; kb += PRODUCERS)
-            tma_load_2d(sbase + kb * rs::A_BLK, am, kb * BK, h * BM, bar(rs::BAR_A_FULL));
+            tma_load_2d_pair(sbase + kb * rs::A_BLK, am, kb * BK, h * BM, lead(rs::BAR_A_FULL));
           ++na;
         }
         for (int kb = 0; kb < p.kblk; ++kb, ++g) {
           const int s = g % rs::STAGES, use = g / rs::STAGES;
-          if (s != pid) continue;
+          if (s % PRODUCERS != pid) continue;
           if (use > 0 && !(ok = mbar_wait(bar(rs::BAR_B_EMPTY + s), (use - 1) & 1, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(rs::BAR_B_FULL + s), rs::B_STAGE);
-          tma_load_2d(sbase + rs::OFF_B + s * rs::B_STAGE, &tm_x, kb * BK, nt * rs::NT, bar(rs::BAR_B_FULL + s));
+          if (rank == 0) mbar_arrive_expect_tx(bar(rs::BAR_B_FULL + s), 2 * rs::B_STAGE);
+          tma_load_2d_pair(sbase + rs::OFF_B + s * rs::B_STAGE, &tm_x, kb * BK, nt * rs::NT + rs::NHALF * rank,
+                           lead(rs::BAR_B_FULL + s));
         }
       }
-      // drain: the releases of this producer's last slot use and of the last A have arrived
-      const int uses = g > pid ? (g - pid + rs::STAGES - 1) / rs::STAGES : 0;
-      if (ok && uses > 0) mbar_wait(bar(rs::BAR_B_EMPTY + pid), (uses - 1) & 1, abort_flag);
+      // drain: the releases of this producer's last slot uses and of the last A have arrived
+      for (int sl = pid; ok && sl < rs::STAGES; sl += PRODUCERS) {
+        const int uses = g > sl ? (g - sl + rs::STAGES - 1) / rs::STAGES : 0;
+        if (uses > 0) ok = mbar_wait(bar(rs::BAR_B_EMPTY + sl), (uses - 1) & 1, abort_flag);
+      }
       if (ok && na > 0) mbar_wait(bar(rs::BAR_A_EMPTY), (na - 1) & 1, abort_flag);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16(BM, rs::NT, false, false);
-    const uint64_t a0 = sdesc_sw128(sbase, 16, 1024);
-    int na = 0, g = 0, lt = 0;
-    bool ok = true;
-    for (int t = t0; t < t1 && ok; ++t, ++lt) {
-      if (batch_start(t)) {
-        if (!(ok = mbar_wait(bar(rs::BAR_A_FULL), na & 1, abort_flag))) break;
-        ++na;
-      }
-      const int buf = lt & 1;
-      if (lt >= 2 && !(ok = mbar_wait(bar(rs::BAR_ACC_EMPTY + buf), ((lt >> 1) - 1) & 1, abort_flag))) break;
-      tc_fence_after();
-      for (int kb = 0; kb < p.kblk; ++kb, ++g) {
-        const int s = g % rs::STAGES;
-        if (!(ok = mbar_wait(bar(rs::BAR_B_FULL + s), (g / rs::STAGES) & 1, abort_flag))) break;
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * BM, rs::NT, false, false);
+      const uint64_t a0 = sdesc_sw128(sbase, 16, 1024);
+      int na = 0, g = 0, lt = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u, ++lt) {
+        if (pair_start(u)) {
+          if (!(ok = mbar_wait(bar(rs::BAR_A_FULL), na & 1, abort_flag))) break;
+          ++na;
+        }
+        const int buf = lt & 1;
+        if (lt >= 2 && !(ok = mbar_wait(bar(rs::BAR_ACC_EMPTY + buf), ((lt >> 1) - 1) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint64_t bd = sdesc_sw128(sbase + rs::OFF_B + s * rs::B_STAGE, 16, 1024);
+        for (int kb = 0; kb < p.kblk; ++kb, ++g) {
+          const int s = g % rs::STAGES;
+          if (!(ok = mbar_wait(bar(rs::BAR_B_FULL + s), (g / rs::STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t bd = sdesc_sw128(sbase + rs::OFF_B + s * rs::B_STAGE, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          tc_mma<1>(tmem + 256 * buf, sdesc_advance(a0, kb * rs::A_BLK + kk * 32), sdesc_advance(bd, kk * 32), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(rs::BAR_B_EMPTY + s));
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma<2>(tmem + 256 * buf, sdesc_advance(a0, kb * rs::A_BLK + kk * 32), sdesc_advance(bd, kk * 32), idesc,
+                      (kb > 0 || kk > 0) ? 1u : 0u);
+          tc_commit_pair(bar(rs::BAR_B_EMPTY + s), 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair(bar(rs::BAR_ACC_FULL + buf), 0x3);
+        if (u + 1 == u1 || (u + 1) % p.n_tiles == 0) tc_commit_pair(bar(rs::BAR_A_EMPTY), 0x3);
       }
-      if (!ok) break;
-      tc_commit(bar(rs::BAR_ACC_FULL + buf));
-      if (t + 1 == t1 || (t + 1) % p.n_tiles == 0) tc_commit(bar(rs::BAR_A_EMPTY));
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if ((warp >= 2 && warp < 6) || warp >= 8) {
     // ----------------------------------------------------------- epilogue
-    const int sp = warp & 3, m = 32 * sp + lane;  // accumulator row = output column m
+    const int sp = warp & 3, m = 32 * sp + lane;  // accumulator row (lane) = output column m of this CTA's head
+    const int cbeg = warp >= 8 ? rs::NT / 2 : 0;  // this warp's half of the tile's columns (tokens)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * sp) << 16);
     griddep_wait();  // outputs are written only once the previous kernel has finished
     int lt = 0;
-    for (int t = t0; t < t1; ++t, ++lt) {
-      const int b = t / p.n_tiles, nt = t % p.n_tiles, buf = lt & 1;
+    for (int u = u0; u < u1; ++u, ++lt) {
+      const int bp = u / p.n_tiles, nt = u % p.n_tiles, b = 2 * bp + static_cast<int>(rank), buf = lt & 1;
       mbar_wait_warp(bar(rs::BAR_ACC_FULL + buf), (lt >> 1) & 1, abort_flag);
       tc_fence_after();
       __nv_bfloat16 *out = (b < p.split ? p.out0 : p.out1) +
                            static_cast<int64_t>(b < p.split ? b : b - p.split) * p.N * BM;
-      for (int c0 = 0; c0 < rs::NT; c0 += 32) {
+      for (int c0 = cbeg; c0 < cbeg + rs::NT / 2; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(lane_addr + 256 * buf + c0, v);
         tmem_wait_ld();
@@ -670,12 +691,22 @@ __global__ void __launch_bounds__(rs::NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(rs::BAR_ACC_EMPTY + buf));
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(bar(rs::BAR_ACC_EMPTY + buf));
+        else mbar_arrive_cluster(mapa_shared(bar(rs::BAR_ACC_EMPTY + buf), 0));
+      }
     }
   }
+  // ---- teardown: both CTAs done with each other's barriers, then free TMEM
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc<1>(tmem, 512);
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(mapa_shared(bar(rs::BAR_EXIT), rank ^ 1));
+    mbar_wait(bar(rs::BAR_EXIT), 0, nullptr);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc<2>(tmem, 512);
 }
 
 // ---------------------------------------------------------- finalizers ----

@@ -903,7 +903,7 @@ mla_status tc_attend_a(const mla_dims *d, const void *qa, const void *W_UK, cons
   __nv_bfloat16 *dsts[2] = {kc, vv};
   {
     CUtensorMap ta0, ta1, tx;
-    if ((s = make_tmap_bf16(&tx, c->data, d->d_c, R, D * 2, 64, G::rs::NT, "cache (c_KV)")) != MLA_OK) return s;
+    if ((s = make_tmap_bf16(&tx, c->data, d->d_c, R, D * 2, 64, G::rs::NHALF, "cache (c_KV)")) != MLA_OK) return s;
     if ((s = make_tmap_bf16(&ta0, W_UK, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UK")) != MLA_OK) return s;
     if ((s = make_tmap_bf16(&ta1, W_UV, d->d_c, HD, d->d_c * 2ull, 64, 128, "W_UV")) != MLA_OK) return s;
     G::rs::Params rp{};
@@ -914,7 +914,7 @@ mla_status tc_attend_a(const mla_dims *d, const void *qa, const void *W_UK, cons
     rp.kblk = d->d_c / G::BK;
     rp.out0 = kc;
     rp.out1 = vv;
-    const int grid = std::max(1, std::min(sm_count(), rp.batches * rp.n_tiles));
+    const int grid = 2 * std::max(1, std::min(sm_count() / 2, (rp.batches / 2) * rp.n_tiles));  // clusters of 2
     if ((s = raise_smem_limit(reinterpret_cast<const void *>(G::k_gemm_resident), SMEM_GEMM_RES, G::rs::SMEM_BYTES,
                               "decompression: set shared memory size")) != MLA_OK)
       return s;
