@@ -80,10 +80,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8 * NUM_BARS);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-  // work item: head, sequence, block of query rows
-  const int h = blockIdx.x % p.n_h;
-  const int b = (blockIdx.x / p.n_h) % p.B;
-  const int qb = blockIdx.x / (p.n_h * p.B);
+  // work item: block of query rows, head, sequence (the query blocks of one
+  // head and sequence are neighbours in the grid, so they run together and
+  // read that head's K_C and V tiles from L2 rather than once each from HBM)
+  const int qb = blockIdx.x % p.qblocks;
+  const int h = (blockIdx.x / p.qblocks) % p.n_h;
+  const int b = blockIdx.x / (p.qblocks * p.n_h);
   const int j0 = qb * QROWS;
 
   if (threadIdx.x == 0) {
