@@ -819,11 +819,14 @@ inline int n_tile_for(int T) {
 
 // Pipeline depth: a launch that fits in one wave runs one CTA per SM and may
 // keep ~200 KB of stages in flight; larger launches fit two CTAs per SM
-// (~100 KB each).
+// (~100 KB each) when three stages fit in that, else one CTA per SM again.
 inline int stages_for(int n_tile, int ctas, int sms) {
-  const int budget = (ctas <= sms ? 200 : 100) * 1024;
-  int s = budget / (A_STAGE + b_stage_bytes(n_tile));
-  const int max_s = ctas <= sms ? 12 : 8;
+  const int stage = A_STAGE + b_stage_bytes(n_tile);
+  // two CTAs per SM only while each still gets three stages; otherwise one
+  // CTA per SM keeps as many stages in flight as ~200 KB allow
+  const bool two = ctas > sms && 3 * stage <= 100 * 1024;
+  int s = (two ? 100 : 200) * 1024 / stage;
+  const int max_s = two ? 8 : 12;
   return s > max_s ? max_s : (s < 3 ? 3 : s);
 }
 

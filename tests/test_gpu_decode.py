@@ -118,6 +118,23 @@ def test_decode_tc_two_queries_causal(mla, orc):
     _run(mla, orc, V2, 15, [2, 64, 65, 66, 1000, 3000], n_q=2)
 
 
+# n_q > 1 runs the kernel whose clusters form one group per query position,
+# each group cutting its own line of rows (rows ordered by query position).
+@pytest.mark.parametrize("n_q, seq_lens", [
+    (3, [3, 257, 4000, 9000, 700]),           # three groups; two clusters left over (74 = 3 x 24 + 2)
+    (2, [5000, 4099, 3001, 12000]),            # long rows cut across the clusters of each group
+    (4, [4, 300, 2000, 65, 128, 129, 6000]),   # four groups, ragged tiles at every edge
+])
+def test_decode_tc_query_position_groups(mla, orc, n_q, seq_lens):
+    _run(mla, orc, V2, 26 + n_q, seq_lens, n_q=n_q)
+
+
+def test_decode_tc_query_position_groups_many_rows(mla, orc):
+    # more rows than clusters in every group: rows finished in place and cut
+    rng = np.random.default_rng(30)
+    _run(mla, orc, V2, 30, list(rng.integers(2, 900, size=160)), n_q=2)
+
+
 def test_decode_tc_bigger_scores_rescale(mla, orc):
     # larger query spread makes the running max move by more than 2^8 and
     # exercises the rescaling of the accumulator
