@@ -25,16 +25,18 @@
 //    in big slots, chunk 8 in the small one; each chunk holds this CTA's 128
 //    tokens as 128 rows so that one N = 256 MMA spans them), then the value
 //    operands of tile i (one big slot per pair of blocks {v, v + 2} and latent
-//    half: 128 of this CTA's latent columns of both). Every ring item costs a commit (~70 ns of tensor-pipe
-//    time), so items are as large as the shared memory allows. Latent columns
+//    half: 128 of this CTA's latent columns of both). Every ring item costs a
+//    commit (~50-70 ns of tensor-pipe time), so items are as large as the
+//    shared memory allows; the small slot is released by the commit that
+//    completes S rather than a commit of its own. Latent columns
 //    are read twice (once per operand), the second time mostly from L2. (An
 //    explicit whole-block L2 prefetch ahead of the score loads measured
 //    slower: it added DRAM reads without removing the score loads' misses.)
-//  * Loads: a TMA instruction occupies its issuing warp for ~0.3 us whatever
-//    the box size (the lanes of a warp issue in parallel), so four producer
-//    warps share the ring, one per big slot: every slot's uses are issued in
-//    order by one warp, whose lanes issue an item's boxes together, and no
-//    slot waits behind another slot's issue.
+//  * Loads: the TMA operations one warp issues complete one after another
+//    (~50 GB/s per warp), those of different warps side by side, so four
+//    producer warps share the ring, one per big slot: every slot's uses are
+//    issued in order by one warp, and no slot waits behind another slot's
+//    loads. Q arrives as three 24 KB boxes from three of the producers.
 //  * P lives in tensor memory, written by the softmax over the scores it was
 //    made from, as the A operand of PV. A pair MMA with M = 128 reads a row's
 //    16-wide K group from both lane m and lane m + 64 (one copy per half of
@@ -55,6 +57,11 @@
 //    With a forced split count S (Params::splits > 0) every row is instead
 //    cut into min(S, its tiles) pieces of near-equal tile counts, and each
 //    cluster takes the pieces that start in its equal share of the tile line.
+//    With n_q > 1 new tokens per sequence (the k_decode<true> instance) the
+//    rows are ordered by query position and, in the automatic plan, each
+//    position's rows are cut by their own group of clusters into ranges of
+//    one length, so the n_q rows of a sequence stream the same cache tiles
+//    at about the same time and all but one read them from L2.
 //  * Rows past a sequence's end: 64-row blocks wholly past it are loaded at
 //    an out-of-range coordinate (TMA zero fill); the one partially valid block
 //    has its value rows past the end zeroed in shared memory before its PV
