@@ -477,24 +477,37 @@ __global__ void __launch_bounds__(ab::NUM_THREADS, 1)
         *reinterpret_cast<uint4 *>(dst) = make_uint4(w0, w1, w2, w3);
       }
     }
-    // q_R,h rows 0..63 (warps of sub-partitions 0, 1): lanes (2k, 2k+1) hold a RoPE pair
-    if (sp < 2) {
-      const bool odd = (row & 1) != 0;
-      for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(lane_addr + p.col_stride + c0, v);
-        tmem_wait_ld();
+    // q_R,h rows 0..63 (warps of sub-partitions 0, 1): lanes (2k, 2k+1) hold a
+    // RoPE pair. The second product overwrites q_R's accumulator, so up to 64
+    // tokens are read into registers first and the shared q_C is released
+    // before they are rotated and stored; larger tiles rotate before release.
+    const bool odd = (row & 1) != 0;
+    auto rotate_store = [&](const uint32_t (&v)[32], int c0) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int t = c0 + c;
-          const float mine = __uint_as_float(v[c]);
-          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-          if (t < p.T) {
-            float x0 = odd ? other : mine, x1 = odd ? mine : other;
-            const float2 cs = rope_tab[t * ab::RPAIRS + (row >> 1)];
-            rope_apply(x0, x1, cs.x, cs.y);
-            p.q[t * q_row + static_cast<int64_t>(head) * (p.d_c + p.d_r) + p.d_c + row] = __float2bfloat16_rn(odd ? x1 : x0);
-          }
+      for (int c = 0; c < 32; ++c) {
+        const int t = c0 + c;
+        const float mine = __uint_as_float(v[c]);
+        const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+        if (t < p.T) {
+          float x0 = odd ? other : mine, x1 = odd ? mine : other;
+          const float2 cs = rope_tab[t * ab::RPAIRS + (row >> 1)];
+          rope_apply(x0, x1, cs.x, cs.y);
+          p.q[t * q_row + static_cast<int64_t>(head) * (p.d_c + p.d_r) + p.d_c + row] = __float2bfloat16_rn(odd ? x1 : x0);
+        }
+      }
+    };
+    const bool early = p.n_tile <= 64;
+    uint32_t qr[2][32];
+    if (sp < 2) {
+      if (early) {
+        tmem_ld32(lane_addr + p.col_stride, qr[0]);
+        if (p.n_tile > 32) tmem_ld32(lane_addr + p.col_stride + 32, qr[1]);
+        tmem_wait_ld();
+      } else {
+        for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+          tmem_ld32(lane_addr + p.col_stride + c0, qr[0]);
+          tmem_wait_ld();
+          rotate_store(qr[0], c0);
         }
       }
     }
@@ -502,6 +515,10 @@ __global__ void __launch_bounds__(ab::NUM_THREADS, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(b2_full);
+    if (sp < 2 && early) {
+      rotate_store(qr[0], 0);
+      if (p.n_tile > 32) rotate_store(qr[1], 32);
+    }
     // q_lat,h: rows 128 mt + row of the second product
     mbar_wait_warp(p2_done, 0, abort_flag);
     tc_fence_after();
