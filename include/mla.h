@@ -135,7 +135,11 @@ mla_status mla_absorb_q(const mla_dims *dims, const void *h, const void *W_DQ, c
  * num_splits (split-KV): 0 = automatic: the tensor-core path concatenates the
  * 256-token KV tiles of all token rows, cuts that line into one equal share
  * per pair of SMs, and merges every row cut by a share boundary with a
- * log-sum-exp combine. S > 0 = forced: every token row is cut into
+ * log-sum-exp combine. With n_q > 1 (and at least n_q pairs of SMs) the pairs
+ * form n_q equal groups, one per query position j; each group cuts the line of
+ * the rows of position j into ranges of one common length, so the n_q rows of
+ * a sequence read the same cache tiles at about the same time (L2 reuse).
+ * S > 0 = forced: every token row is cut into
  * min(S, its tiles) pieces of near-equal tile counts (S = 1: no split), each
  * pair of SMs takes the pieces that start in its equal share of the tile line,
  * and rows of more than one piece are merged by the same combine. The
