@@ -48,6 +48,14 @@ MUTANTS = [
     ("merged absorption drops the last head row",
      "        for (int i = 0; i < p->d_h; ++i)\n          acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ",
      "        for (int i = 0; i < p->d_h - 1; ++i)\n          acc += W_UK[((int64_t)hh * p->d_h + i) * p->d_c + j] * W_UQ"),
+    ("order A decompresses values with W_UK",
+     "        orc_matvec(Wv, p->d_h, p->d_c, ckv, v);", "        orc_matvec(Wk, p->d_h, p->d_c, ckv, v);"),
+    ("order A reads every head's values from head 0",
+     "const double *Wv = W_UV + hh * (int64_t)p->d_h * p->d_c;", "const double *Wv = W_UV;"),
+    ("order A drops the RoPE term",
+     "          acc += qr[jj] * orc_read(c->data, c->dtype, row * D + p->d_c + jj);",
+     "          acc += 0.0 * qr[jj];"),
+    ("order A softmax not normalised", "double w = exp(scores[i] - m) / z;", "double w = exp(scores[i] - m);"),
     ("output projection skips a token row",
      "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)t * cols, y + (int64_t)t * rows);",
      "for (int t = 0; t < T; ++t) orc_matvec(W, rows, cols, x + (int64_t)(t > 0 ? t - 1 : 0) * cols, y + (int64_t)t * rows);"),

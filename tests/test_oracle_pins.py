@@ -203,6 +203,34 @@ def test_mla_reduces_to_mha(orc):
     assert np.allclose(o, ref.numpy().reshape(n_h, d_h), rtol=1e-12, atol=1e-13)
 
 
+def test_order_a_is_sdpa_over_decompressed_heads(orc):
+    # Order A (walk-through, section 3: decompress, then dot) is ordinary
+    # multi-head attention: per head, keys [W_UK,h c_KV,i ; k_R,i] with the
+    # RoPE key shared by all heads, values W_UV,h c_KV,i, query [q_C,h ; q_R,h],
+    # scale 1/sqrt(d_h + d_R). Reference: numpy decompression, torch SDPA, fp64.
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(14)
+    n_h, d_h, d_c, d_r = 3, 4, 8, 2
+    p = orc.dims(d=8, n_h=n_h, d_h=d_h, d_c=d_c, d_cq=8, d_r=d_r)
+    lens = (11, 6)
+    L = max(lens)
+    rows = rng.standard_normal((len(lens), L, d_c + d_r))
+    W_UK = rng.standard_normal((n_h * d_h, d_c))
+    W_UV = rng.standard_normal((n_h * d_h, d_c))
+    q_C = rng.standard_normal((len(lens), n_h, d_h))
+    q_R = rng.standard_normal((len(lens), n_h, d_r))
+    o = orc.decode_order_a(p, q_C, q_R, W_UK, W_UV, orc.Cache(rows), np.array(lens, np.int32), 1)
+    for b, n in enumerate(lens):
+        ckv, k_r = rows[b, :n, :d_c], rows[b, :n, d_c:]
+        for hh in range(n_h):
+            K = np.concatenate([ckv @ W_UK[hh * d_h:(hh + 1) * d_h].T, k_r], 1)
+            V = ckv @ W_UV[hh * d_h:(hh + 1) * d_h].T
+            Q = np.concatenate([q_C[b, hh], q_R[b, hh]])[None]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.tensor(Q), torch.tensor(K), torch.tensor(V), scale=1 / math.sqrt(d_h + d_r))
+            assert np.allclose(o[b, hh], ref.numpy()[0], rtol=1e-12, atol=1e-13)
+
+
 def test_split_kv_combine_equals_unsplit(orc):
     rng = np.random.default_rng(7)
     p = orc.dims(d=8, n_h=1, d_h=4, d_c=16, d_cq=8, d_r=4)
