@@ -114,20 +114,58 @@ def cache_copies(cache_bytes):
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons, each stamped with the
-    host time it arrived, so that the summary keeps only the samples taken while
-    the timed region ran (mark() brackets it). The GPU is addressed by UUID,
-    which stays right under CUDA_VISIBLE_DEVICES."""
+    """Samples of SM clock and throttle reasons, each stamped with the host time
+    it was taken, so that the summary keeps only the samples taken while the
+    timed region ran (mark() brackets it). NVML is read in-process every ~2 ms
+    (read-only queries), so that even a timed region of a few tens of
+    milliseconds holds a dozen samples; without NVML, nvidia-smi is polled every
+    20 ms instead. Both record the same fields in the same line format. The GPU
+    is addressed by UUID, which stays right under CUDA_VISIBLE_DEVICES."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id):
+    PERIOD_S = 0.002  # NVML polling period
+
+    def __init__(self, gpu_id, nvml=None):
         self.gpu = gpu_id
         self.proc = None
+        self.poller = None
+        self.stop = threading.Event()
+        self.nvml = nvml  # the pynvml module (injectable for tests); None: import it
         self.samples = []  # (host time, line)
         self.window = None
+
+    def _nvml_handle(self):
+        nv = self.nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        try:
+            g = str(self.gpu)
+            h = nv.nvmlDeviceGetHandleByUUID(g) if g.startswith("GPU-") else nv.nvmlDeviceGetHandleByIndex(int(g))
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:
+            nv.nvmlShutdown()
+            raise
+        self.nvml = nv
+        return h, smax
+
+    def _poll(self, h, smax):
+        nv = self.nvml
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+            except Exception:
+                break
+            flags = ", ".join("Active" if mask & b else "Not Active" for b in bits)
+            self.samples.append((time.perf_counter(), f"0, {sm}, {smax}, {watts:.2f}, {mask:#x}, {flags}\n"))
+            self.stop.wait(self.PERIOD_S)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -135,6 +173,22 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), line))
 
     def __enter__(self):
+        try:
+            h, smax = self._nvml_handle()
+        except Exception:
+            h = None
+        if h is not None:
+            self.poller = threading.Thread(target=self._poll, args=(h, smax), daemon=True)
+            self.poller.start()
+            t0 = time.perf_counter()
+            while not self.samples and time.perf_counter() - t0 < 5.0 and self.poller.is_alive():
+                time.sleep(0.001)
+            if self.samples:
+                return self
+            self.stop.set()  # NVML answered the set-up but not the queries: fall back to nvidia-smi
+            self.poller.join(timeout=5)
+            self.poller = None
+            self.nvml.nvmlShutdown()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -153,6 +207,13 @@ class ClockSampler:
         self.window = (t_begin, t_end)
 
     def __exit__(self, *a):
+        if self.poller is not None:
+            self.stop.set()
+            self.poller.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -168,7 +229,7 @@ class ClockSampler:
         if self.window is not None:
             a, b = self.window
             inside = [x for x in lines if a <= x[0] <= b]
-            # a short timed region may fall between two 20 ms samples: keep the nearest one
+            # a timed region shorter than the sampling period may hold no sample: keep the nearest one
             lines = inside or sorted(lines, key=lambda x: abs(x[0] - 0.5 * (a + b)))[:1]
         for _, l in lines:
             parts = [x.strip() for x in l.split(",")]

@@ -1,10 +1,13 @@
 """Host-side pieces of bench.py, on CPU: the clock summary keeps only the
 samples of the timed region and reports every throttle reason it saw; the
+in-process NVML sampler (driven here by a fake NVML module, read-only
+queries) feeds the same summary and falls back when NVML fails; the
 DRAM traffic figure is taken from the committed profile only while the
 profiled source is unchanged; the reported config names the workload."""
 import hashlib
 import os
 import sys
+import time
 
 import numpy as np
 
@@ -76,3 +79,67 @@ def test_percentiles_of_step_durations():
     ms = [0.1 * k for k in range(1, 101)]  # 0.1 .. 10 ms
     p10, p50, p90 = bench.percentiles_us(ms)
     assert abs(p10 - 1090.0) < 1e-6 and abs(p50 - 5050.0) < 1e-6 and abs(p90 - 9010.0) < 1e-6
+
+
+class _FakeNVML:
+    """The few read-only NVML entry points the sampler calls, with made-up
+    reason bits; counts init/shutdown so that the test sees them paired."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 1 << 0
+    nvmlClocksEventReasonHwThermalSlowdown = 1 << 1
+    nvmlClocksEventReasonSwThermalSlowdown = 1 << 2
+    nvmlClocksEventReasonSwPowerCap = 1 << 3
+
+    def __init__(self, fail_queries=False):
+        self.fail_queries = fail_queries
+        self.inits = self.shutdowns = self.queries = 0
+        self.handle_of = None
+
+    def nvmlInit(self):
+        self.inits += 1
+
+    def nvmlShutdown(self):
+        self.shutdowns += 1
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        self.handle_of = uuid
+        return "h"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        self.handle_of = i
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        assert h == "h" and kind == self.NVML_CLOCK_SM
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        if self.fail_queries:
+            raise RuntimeError("not supported")
+        self.queries += 1
+        return 1965 if self.queries % 2 else 1950
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.nvmlClocksEventReasonSwPowerCap
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 700000  # milliwatts
+
+
+def test_nvml_sampler_fills_the_timed_window():
+    fake = _FakeNVML()
+    with bench.ClockSampler("GPU-0000", nvml=fake) as c:
+        a = time.perf_counter()
+        time.sleep(0.04)
+        c.mark(a, time.perf_counter())
+    assert fake.handle_of == "GPU-0000" and fake.inits == 1 and fake.shutdowns == 1
+    s = c.summary()
+    assert s["samples"] >= 5 and s["sm_max_mhz"] == 1965.0
+    assert 1950.0 <= s["sm_mhz"] <= 1965.0 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_nvml_sampler_falls_back_when_queries_fail():
+    fake = _FakeNVML(fail_queries=True)
+    with bench.ClockSampler("3", nvml=fake) as c:
+        assert c.poller is None  # handed over to the nvidia-smi path
+    assert fake.handle_of == 3 and fake.inits == 1 and fake.shutdowns == 1
