@@ -25,7 +25,7 @@
  *  - "Attention / RoPE tutorial" (xianlaiwan.cn): RoPE rotates q and k by
  *    position so that scores depend on the relative offset (RoFormer).
  *
- * Readings taken where the pages are silent (each listed in the design notes):
+ * Readings taken where the pages are silent:
  *  - softmax scale 1/sqrt(d_h + d_R) (the score lives in the 192-d
  *    concatenated space of step 4);
  *  - RoPE pairs are interleaved (2i, 2i+1), theta_i = base^(-2i/d_R);
@@ -35,8 +35,24 @@
  *  - no normalisation layers and no biases.
  *
  * Parity pins (tests/test_oracle_pins.py): every function below is pinned by
- * at least one check that does not re-run this code's own formula. See the
- * pin table in the design notes.
+ * at least one check that does not re-run this code's own formula:
+ *  - orc_rope: the d_R = 2 closed form at position 1, the theta table, norm
+ *    preservation, RoPE(x, 0) = x and the relative-position property;
+ *  - orc_slot: hand-computed slots, paged = contiguous on the same rows;
+ *  - orc_append, orc_absorb_q: the same chains through torch.matmul in fp64,
+ *    RoPE shift invariance end to end, and (absorb) the merged matrix;
+ *  - orc_decode (orc_attend_latent, orc_visible): worked examples computed by
+ *    hand (tests/golden/hand_examples.json), one cached row, identical rows,
+ *    q = 0, causal masking within a step, the reduction to torch's
+ *    scaled-dot-product attention, order A = order B;
+ *  - orc_attend_range, orc_combine: any split merged equals the unsplit result;
+ *  - orc_out_proj, orc_o_proj, orc_absorb_wo, orc_absorb_merge: library
+ *    products, and each absorbed form against its two-stage form;
+ *  - orc_decode_order_a: order A = order B, and torch's scaled-dot-product
+ *    attention over heads decompressed by numpy;
+ *  - bf16 reads: exact values.
+ * tests/test_oracle_mutants.py plants plausible mistakes in a copy of this
+ * file, one at a time, and requires a pin to fail against each.
  */
 #include <math.h>
 #include <stdint.h>
