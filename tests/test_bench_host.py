@@ -143,3 +143,20 @@ def test_nvml_sampler_falls_back_when_queries_fail():
     with bench.ClockSampler("3", nvml=fake) as c:
         assert c.poller is None  # handed over to the nvidia-smi path
     assert fake.handle_of == 3 and fake.inits == 1 and fake.shutdowns == 1
+
+
+def test_profile_summaries_leave_clocks_alone_and_parse():
+    """Every ncu command a summary records runs with --clock-control none, and
+    each decode summary carries the two fields the bench reads."""
+    pdir = os.path.join(ROOT, "profiles")
+    for name in sorted(os.listdir(pdir)):
+        text = open(os.path.join(pdir, name)).read()
+        # an ncu command may continue over backslash-ended lines
+        cmds = text.replace("\\\n", " ").splitlines()
+        for c in cmds:
+            if c.lstrip().startswith("ncu "):
+                assert "--clock-control none" in c, (name, c)
+        if name.startswith("k_decode_"):
+            fields = dict(l.split(": ", 1) for l in text.splitlines()
+                          if l.startswith(("traffic_bytes_per_launch:", "decode_source_sha256_16:")))
+            assert int(fields["traffic_bytes_per_launch"]) > 0 and len(fields["decode_source_sha256_16"].strip()) == 16
